@@ -1,0 +1,195 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged KV-cache decode attention for NVIDIA B200
+ * (sm_100a).  Hand-written CUDA kernels behind plain pointers and sizes.
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - Pointers named key/value/cache/q/out/tables/lens/pairs/workspace/dev_err
+ *    are DEVICE pointers on the current CUDA device.  The caller owns every
+ *    buffer (the workspace and the error word included).  The library
+ *    allocates nothing, keeps no pointer after returning and holds no state
+ *    that changes results; it is safe to call from several host threads.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  Results are ready once the stream reaches the
+ *    point of the call.
+ *  - Host-side errors (null pointer, bad size, unsupported shape, short
+ *    workspace, failed launch) are returned synchronously as a pa_status and
+ *    nothing is launched.
+ *  - Data-dependent errors are found on the device: the offending entry is
+ *    skipped (its tokens take no part in the result, the write or copy does
+ *    not happen) and a PA_DEVERR_* bit is OR-ed into *dev_err.  dev_err may be
+ *    NULL (errors are then only skipped).  Read it after synchronising.  No
+ *    kernel ever traps; every wait inside a kernel is bounded and sets
+ *    PA_DEVERR_TIMEOUT if it runs out.
+ *
+ * Data layout
+ * -----------
+ *  Pool ("physical KV blocks"):  k_cache, v_cache  [num_blocks][num_kv_heads][block_size][head_dim]
+ *  New tokens:                   key, value        [num_tokens][num_kv_heads][head_dim]
+ *  Queries / outputs:            q, out            [num_seqs][num_heads][head_dim]
+ *  Block tables:                 int32 [num_seqs][max_blocks_per_seq]; entry i of row s is the
+ *                                physical block of logical block i (tokens [i*B, (i+1)*B)).
+ *  Context lengths:              int32 [num_seqs], the number of tokens each query attends to,
+ *                                the token written this step included.
+ *  All arrays are dense and row-major; data pointers must be 16-byte aligned.
+ *  Query heads [h*g, (h+1)*g) share kv head h, g = num_heads / num_kv_heads.
+ *
+ * Sources: "PagedAttention blog" (0539edu.com) section 3(3) (logical blocks of
+ * B tokens, the block table, filled slots, the decode-time gather) and section
+ * 4 (parallel samples sharing blocks, copy-on-write); "Month 2 · PagedAttention"
+ * study guide (weishuz.com) section 02 (mapping table), section 03 reading 4
+ * (block_table and slot_mapping handed to the attention kernel) and section 06
+ * (the kernel is ordinary attention that gathers K and V from non-contiguous
+ * addresses).  The pages print no formula; the attention computed is
+ * softmax(scale * q . K^T) . V over the sequence's context.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_dtype {
+    PA_F32 = 0,   /* IEEE fp32 */
+    PA_BF16 = 1   /* bfloat16 */
+} pa_dtype;
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null pointer, negative or zero size, misaligned pointer,
+                                 num_heads not a multiple of num_kv_heads, ... */
+    PA_ERR_UNSUPPORTED = 2,   /* head_dim not in {64, 128}, block_size not in {4, 8, 16, 32},
+                                 partition_size not a positive multiple of 32 (or > 8192),
+                                 dtype combination not offered */
+    PA_ERR_WORKSPACE = 3,     /* workspace_bytes below pa_decode_workspace_bytes() */
+    PA_ERR_CUDA = 4           /* a CUDA runtime call or a kernel launch failed */
+} pa_status;
+
+/* Bits OR-ed into *dev_err by the kernels. */
+#define PA_DEVERR_BLOCK_ID 0x1  /* a block-table entry needed for the context is outside [0, num_blocks) */
+#define PA_DEVERR_SLOT     0x2  /* a slot_mapping entry is >= num_blocks * block_size */
+#define PA_DEVERR_CONTEXT  0x4  /* a context length is < 0 or above the capacity (clamped to it) */
+#define PA_DEVERR_COPY     0x8  /* a copy pair names a block outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT  0x10 /* a bounded wait for an asynchronous copy ran out */
+
+typedef void* pa_stream;        /* a cudaStream_t */
+
+/*
+ * pa_reshape_and_cache -- write each new token's K and V into its slot of the
+ * pool ("Month 2 · PagedAttention" section 03 reading 4: slot_mapping says
+ * where each token's K/V go; "PagedAttention blog" section 3(3): the K/V are
+ * filled into the physical blocks through the mapping).
+ *
+ *   key, value    [num_tokens][num_kv_heads][head_dim] of `dtype`, read only
+ *   k_cache, v_cache  the pool, [num_blocks][num_kv_heads][block_size][head_dim] of `dtype`
+ *   slot_mapping  int64 [num_tokens]: token t goes to block slot/block_size at offset
+ *                 slot%block_size, for every kv head.  slot < 0: no write.
+ *                 slot >= num_blocks*block_size: no write, PA_DEVERR_SLOT.
+ * The copy is bit-exact.  Two tokens naming the same slot race (caller error).
+ * num_tokens == 0 is a no-op.
+ */
+int pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                         int32_t* dev_err, pa_stream stream);
+
+/*
+ * pa_decode_workspace_bytes -- bytes of device workspace pa_decode needs for
+ * a batch of num_seqs sequences whose contexts do not exceed max_context_len,
+ * split into partitions of partition_size tokens.  Returns 0 on bad arguments.
+ * The workspace holds the per-call work list (num_seqs * ceil(max_context_len /
+ * partition_size) entries) and, when a context can span several partitions,
+ * one (max, sum, unnormalised output) partial per sequence, head and partition
+ * in fp32.  Its contents need no initialisation.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                 int max_context_len, int partition_size);
+
+/*
+ * pa_decode -- decode attention of each sequence's query against the K/V of
+ * its context, gathered through its block table ("PagedAttention blog"
+ * section 3(3) decode step; "Month 2 · PagedAttention" section 06).
+ *
+ *   out           [num_seqs][num_heads][head_dim] of `out_dtype` (PA_F32, or equal to `dtype`)
+ *   q             [num_seqs][num_heads][head_dim] of `dtype`
+ *   k_cache, v_cache  the pool of `dtype` (PA_F32 or PA_BF16)
+ *   block_tables  int32 [num_seqs][max_blocks_per_seq]; entries past ceil(ctx/block_size)
+ *                 are never read (may be -1).  Slots past ctx in the last block (the
+ *                 reservation) are never used, whatever they hold (NaN included).
+ *   context_lens  int32 [num_seqs]; 0 gives a zero output row.
+ *   max_context_len  host-side bound on every context length; 0 means
+ *                 max_blocks_per_seq * block_size.  Longer contexts are clamped to
+ *                 min(max_context_len, max_blocks_per_seq * block_size) and flagged.
+ *   scale         logits are scale * (q . k)
+ *   partition_size  contexts are cut into partitions of this many tokens, processed in
+ *                 parallel and merged in partition order by a second kernel (512 is the
+ *                 usual choice).  Must be a multiple of 32 and of block_size, <= 8192.
+ *   workspace     at least pa_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+ *                 max_context_len, partition_size) bytes, 256-byte aligned.
+ * Arithmetic: fp32 accumulation.  bf16 inputs: q.K products exact, softmax weights
+ * carried to about 16 significant bits into the value product; fp32 inputs: fp32
+ * throughout.  The result depends only on the logical order of the tokens, so it is
+ * bit-identical under any renumbering of physical blocks and run to run.
+ * Launches three kernels (plan, attention, merge) on `stream`.
+ */
+int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+              const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+              int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+              int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+              int partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+              int32_t* dev_err, pa_stream stream);
+
+/*
+ * pa_decode_phases -- pa_decode split into its three launches, selected by the
+ * bit mask `phases` (PA_PHASE_*; PA_PHASE_ALL gives pa_decode).  The plan
+ * depends only on context_lens, the shapes and partition_size, so a caller
+ * running several layers over the same batch may plan once and run
+ * ATTEND|REDUCE per layer with the same workspace; a caller timing the
+ * attention kernel alone brackets the ATTEND call with its own events.
+ * Phases must run in order PLAN, ATTEND, REDUCE on the same workspace.
+ * Arguments as for pa_decode.
+ */
+#define PA_PHASE_PLAN   0x1
+#define PA_PHASE_ATTEND 0x2
+#define PA_PHASE_REDUCE 0x4
+#define PA_PHASE_ALL    0x7
+int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, int num_seqs, int num_heads,
+                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                     int max_blocks_per_seq, int max_context_len, float scale,
+                     int partition_size, void* workspace, size_t workspace_bytes,
+                     pa_dtype dtype, int32_t* dev_err, pa_stream stream, int phases);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copies ("PagedAttention blog" section 4,
+ * step 2: the writer gets a new physical block holding a copy of the shared one).
+ *
+ *   k_cache, v_cache  the pool
+ *   src_dst_pairs int64 [num_pairs][2] (device): whole block src (all kv heads, all
+ *                 slots) is copied over block dst, in both pools.  Destinations must be
+ *                 pairwise distinct and no destination may also be a source of the same
+ *                 call (otherwise the result is undefined).  A pair naming a block
+ *                 outside [0, num_blocks) is skipped and flagged PA_DEVERR_COPY.
+ *   block_bytes   bytes of one block of one pool: num_kv_heads*block_size*head_dim*element
+ *                 size; a positive multiple of 16.
+ * The copy is bit-exact.  num_pairs == 0 is a no-op.
+ */
+int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
+                   size_t block_bytes, int num_blocks, int32_t* dev_err, pa_stream stream);
+
+/* Human-readable name of a pa_status value (static storage). */
+const char* pa_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* PA_H_ */

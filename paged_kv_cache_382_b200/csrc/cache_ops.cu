@@ -1,0 +1,132 @@
+// cache_ops.cu -- writes into the paged KV pool:
+//   pa_reshape_and_cache: scatter of each new token's K/V into its slot
+//     ("Month 2 · PagedAttention", section 03 reading 4: slot_mapping tells the
+//     kernel where each token's K/V go; "PagedAttention blog", section 3(3)).
+//   pa_copy_blocks: whole-block copies for copy-on-write ("PagedAttention
+//     blog", section 4 step 2).
+// Both are plain 16-byte vector copies: bit-exact, coalesced, HBM/latency bound.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+// One CTA per new token.  A token's K (and V) for all kv heads is
+// num_kv_heads rows of `row_vecs` 16-byte vectors; row h goes to
+// cache[block][h][offset][:].
+__global__ void __launch_bounds__(256)
+reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                         uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                         const int64_t* __restrict__ slot_mapping, int num_kv_heads, int row_vecs,
+                         int block_size, int64_t num_slots, int32_t* dev_err) {
+    const int t = blockIdx.x;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0) flag_error(dev_err, PA_DEVERR_SLOT);
+        return;
+    }
+    const int64_t block = slot / block_size;
+    const int offset = static_cast<int>(slot - block * block_size);
+    const int per_token = num_kv_heads * row_vecs;
+    const uint4* ksrc = key + static_cast<int64_t>(t) * per_token;
+    const uint4* vsrc = value + static_cast<int64_t>(t) * per_token;
+    for (int i = threadIdx.x; i < per_token; i += blockDim.x) {
+        const int h = i / row_vecs;
+        const int v = i - h * row_vecs;
+        const int64_t dst = ((block * num_kv_heads + h) * block_size + offset) * row_vecs + v;
+        k_cache[dst] = ksrc[i];
+        v_cache[dst] = vsrc[i];
+    }
+}
+
+// grid.y = pair index; grid.x CTAs stride over the block's 16-byte vectors.
+__global__ void __launch_bounds__(256)
+copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                   const int64_t* __restrict__ pairs, int64_t block_vecs, int num_blocks,
+                   int32_t* dev_err) {
+    const int64_t src = pairs[2 * static_cast<int64_t>(blockIdx.y)];
+    const int64_t dst = pairs[2 * static_cast<int64_t>(blockIdx.y) + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(dev_err, PA_DEVERR_COPY);
+        return;
+    }
+    const uint4* ks = k_cache + src * block_vecs;
+    const uint4* vs = v_cache + src * block_vecs;
+    uint4* kd = k_cache + dst * block_vecs;
+    uint4* vd = v_cache + dst * block_vecs;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < block_vecs;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 a = ks[i];
+        const uint4 b = vs[i];
+        kd[i] = a;
+        vd[i] = b;
+    }
+}
+
+}  // namespace pa
+
+extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                                    void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                    int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                    pa_dtype dtype, int32_t* dev_err, pa_stream stream) {
+    using namespace pa;
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0 || !valid_dtype(dtype))
+        return PA_ERR_INVALID_ARG;
+    if (!(head_dim == 64 || head_dim == 128)) return PA_ERR_UNSUPPORTED;
+    if (!(block_size == 4 || block_size == 8 || block_size == 16 || block_size == 32))
+        return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned_to(key, 16) || !aligned_to(value, 16) || !aligned_to(k_cache, 16) ||
+        !aligned_to(v_cache, 16) || !aligned_to(slot_mapping, 8))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens > 2147483647 / 2) return PA_ERR_INVALID_ARG;
+    const int row_vecs = head_dim * element_bytes(dtype) / 16;
+    const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+    const int per_token = num_kv_heads * row_vecs;
+    const int threads = per_token >= 256 ? 256 : ((per_token + 31) / 32) * 32;
+    reshape_and_cache_kernel<<<num_tokens, threads, 0, as_stream(stream)>>>(
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(k_cache),
+        static_cast<uint4*>(v_cache), slot_mapping, num_kv_heads, row_vecs, block_size, num_slots,
+        dev_err);
+    return launch_status();
+}
+
+extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,
+                              int num_pairs, size_t block_bytes, int num_blocks, int32_t* dev_err,
+                              pa_stream stream) {
+    using namespace pa;
+    if (num_pairs < 0 || num_blocks <= 0 || block_bytes == 0 || block_bytes % 16 != 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !src_dst_pairs) return PA_ERR_INVALID_ARG;
+    if (!aligned_to(k_cache, 16) || !aligned_to(v_cache, 16) || !aligned_to(src_dst_pairs, 8))
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs > 65535) return PA_ERR_UNSUPPORTED;   // grid.y limit
+    const int64_t block_vecs = static_cast<int64_t>(block_bytes / 16);
+    const int threads = 256;
+    int64_t ctas = (block_vecs + threads * 4 - 1) / (threads * 4);
+    if (ctas < 1) ctas = 1;
+    if (ctas > 1024) ctas = 1024;
+    dim3 grid(static_cast<unsigned>(ctas), static_cast<unsigned>(num_pairs));
+    copy_blocks_kernel<<<grid, threads, 0, as_stream(stream)>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), src_dst_pairs, block_vecs,
+        num_blocks, dev_err);
+    return launch_status();
+}
+
+extern "C" const char* pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: invalid argument";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: shape or dtype not supported";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace too small";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA call or kernel launch failed";
+        default: return "unknown pa_status";
+    }
+}
+
+extern "C" int pa_version(void) { return 100; }

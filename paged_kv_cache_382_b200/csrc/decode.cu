@@ -1,0 +1,864 @@
+// decode.cu -- paged decode attention on B200 (sm_100a).
+//
+// What is computed ("PagedAttention blog", section 3(3) decode step;
+// "Month 2 · PagedAttention", section 06): for every sequence s and query head
+// h, ordinary attention softmax(scale * q . K^T) . V over the sequence's
+// context_len tokens, whose K/V rows are found through the block table
+// (logical block i -> physical block table[s][i]; token j is slot j % B of
+// logical block j / B).  Slots past the context in the last block are never
+// used.
+//
+// How (three launches on the caller's stream):
+//   1. plan:    one CTA turns context_lens into a work list of (seq, partition)
+//               items, whole partitions first, ragged tails last.
+//   2. attend:  persistent CTAs take (item, kv head, head group) units in a
+//               static stride.  One unit = one partition of up to
+//               partition_size tokens of one kv head, for the (up to 8) query
+//               heads that share it, so each K/V byte is read once per group.
+//               bf16: each warp streams 16-token tiles of K and V through its
+//               own ring of shared-memory stages, filled by tensor-map bulk
+//               copies (128-byte swizzle) completing on mbarriers; q.K^T and
+//               p.V run on the tensor cores (m16n8k16, tokens as M, the query
+//               heads as N) with an online softmax in fp32 registers.
+//               fp32: a plain CUDA-core warp-per-token loop.
+//               A sequence that fits one partition writes its output directly;
+//               otherwise each partition writes (max, sum, unnormalised
+//               output) to the workspace.
+//   3. reduce:  merges the partitions of each (seq, head) in partition order.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <climits>
+#include <cmath>
+
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+constexpr float NEG_INF = -INFINITY;
+constexpr float LOG2E = 1.4426950408889634f;
+// Lazy rescaling: the running max of a head is only raised when a tile's max
+// exceeds it by more than this many powers of two, so most tiles skip the
+// rescale of the accumulators.  Weights stay <= 2^8 -- harmless in fp32 and
+// exact-range in bf16; the final quotient is unchanged.
+constexpr float RESCALE_THRESHOLD = 8.0f;
+
+struct DecodeArgs {
+    void* out;
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    int32_t* dev_err;
+    int* ws_count;       // [1]   number of work items
+    int* ws_items;       // [num_seqs * max_parts]  item = seq * max_parts + partition
+    float2* ws_ml;       // [num_seqs][num_heads][max_parts]  (log2-domain max, sum)
+    float* ws_acc;       // [num_seqs][num_heads][max_parts][head_dim]
+    int num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks;
+    int cap;             // contexts are clamped to [0, cap]
+    int partition_size;
+    int max_parts;       // ceil(cap / partition_size), at least 1
+    int group;           // query heads per kv head
+    int head_groups;     // ceil(group / 8): units per kv head
+    float scale_log2;    // scale * log2(e)
+    int out_f32;         // 1: out is fp32, 0: out is bf16
+};
+
+__device__ __forceinline__ int clamp_context(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
+
+// ---------------------------------------------------------------------------
+// 1. plan
+// ---------------------------------------------------------------------------
+
+constexpr int PLAN_THREADS = 1024;
+
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(FULL_MASK, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+
+// Exclusive prefix sum of v over the CTA; *total receives the sum.
+// `scratch` holds 33 ints.
+__device__ int cta_exclusive_scan(int v, int* total, int* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int inc = warp_inclusive_scan(v);
+    __syncthreads();
+    if (lane == 31) scratch[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int x = lane < nw ? scratch[lane] : 0;
+        const int xi = warp_inclusive_scan(x);
+        if (lane < nw) scratch[lane] = xi - x;
+        if (lane == 31) scratch[32] = xi;
+    }
+    __syncthreads();
+    *total = scratch[32];
+    return scratch[warp] + inc - v;
+}
+
+__global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
+    __shared__ int scratch[33];
+    const int P = a.partition_size;
+    int nf = 0, nt = 0;
+    bool bad = false;
+    for (int s = threadIdx.x; s < a.num_seqs; s += PLAN_THREADS) {
+        const int raw = a.context_lens[s];
+        const int c = clamp_context(raw, a.cap);
+        bad |= (c != raw);
+        nf += c / P;
+        nt += (c % P) != 0;
+    }
+    if (bad) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
+    int full_total = 0, tail_total = 0;
+    cta_exclusive_scan(nf, &full_total, scratch);
+    cta_exclusive_scan(nt, &tail_total, scratch);
+    int base_full = 0, base_tail = full_total;
+    for (int start = 0; start < a.num_seqs; start += PLAN_THREADS) {
+        const int s = start + threadIdx.x;
+        int f = 0, t = 0;
+        if (s < a.num_seqs) {
+            const int c = clamp_context(a.context_lens[s], a.cap);
+            f = c / P;
+            t = (c % P) != 0;
+        }
+        int chunk_f = 0, chunk_t = 0;
+        const int ef = cta_exclusive_scan(f, &chunk_f, scratch);
+        const int et = cta_exclusive_scan(t, &chunk_t, scratch);
+        for (int k = 0; k < f; ++k) a.ws_items[base_full + ef + k] = s * a.max_parts + k;
+        if (t) a.ws_items[base_tail + et] = s * a.max_parts + f;
+        base_full += chunk_f;
+        base_tail += chunk_t;
+    }
+    if (threadIdx.x == 0) *a.ws_count = full_total + tail_total;
+}
+
+// ---------------------------------------------------------------------------
+// shared epilogue: merge the W warps' partial softmax states of one unit and
+// store the output row (single partition) or the partition's partial.
+// mm, ml: [W][8] running max (log2 domain) and sum; mo: [W][8][D].
+// ---------------------------------------------------------------------------
+
+template <int W, int D>
+__device__ __forceinline__ void combine_store(const DecodeArgs& a, const float* mm, const float* ml,
+                                              const float* mo, int s, int p, int nparts, int head0,
+                                              int gsub) {
+    for (int idx = threadIdx.x; idx < gsub * D; idx += W * 32) {
+        const int n = idx / D, d = idx - (idx / D) * D;
+        float M = NEG_INF;
+#pragma unroll
+        for (int w = 0; w < W; ++w) M = fmaxf(M, mm[w * 8 + n]);
+        float L = 0.f, O = 0.f;
+        if (M != NEG_INF) {
+#pragma unroll
+            for (int w = 0; w < W; ++w) {
+                const float e = exp2_approx(mm[w * 8 + n] - M);
+                L += e * ml[w * 8 + n];
+                O += e * mo[(w * 8 + n) * D + d];
+            }
+        }
+        const size_t row = static_cast<size_t>(s) * a.num_heads + head0 + n;
+        if (nparts == 1) {
+            const float v = L > 0.f ? O / L : 0.f;
+            if (a.out_f32)
+                static_cast<float*>(a.out)[row * D + d] = v;
+            else
+                static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(v);
+        } else {
+            const size_t slot = row * a.max_parts + p;
+            a.ws_acc[slot * D + d] = O;
+            if (d == 0) a.ws_ml[slot] = make_float2(M, L);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2a. attend, bf16: tensor-map bulk copies into per-warp stage rings + warp MMA
+// ---------------------------------------------------------------------------
+
+// Shared-memory geometry of one 16-token tile.  A K (or V) tile is stored as
+// D/64 "halves" of 64 columns (128 bytes per row) in the 128-byte swizzled
+// layout the bulk copy produces: inside each 1024-byte span, the 16-byte chunk
+// c of row r sits at chunk c ^ (r % 8).  A tile is filled by 16/RB boxes of RB
+// rows (RB = min(block_size, 16)); boxes start on 1024-byte boundaries.
+template <int D, int RB>
+struct TileGeom {
+    static constexpr int NH = D / 64;
+    static constexpr int BOXES = 16 / RB;
+    static constexpr int BOX_STRIDE = RB * 128 >= 1024 ? RB * 128 : 1024;
+    static constexpr int HALF = BOXES * BOX_STRIDE;   // bytes of one 64-column half
+    static constexpr int STAGE = 2 * NH * HALF;       // K halves, then V halves
+    __host__ __device__ static constexpr uint32_t row_off(int r) {
+        return static_cast<uint32_t>((r / RB) * BOX_STRIDE + (r % RB) * 128);
+    }
+};
+
+template <int D, int RB, int W, int NS>
+__global__ void __launch_bounds__(W * 32)
+attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const DecodeArgs a) {
+    using Geo = TileGeom<D, RB>;
+    constexpr int NH = Geo::NH, KS = D / 16, HALF = Geo::HALF, STAGE = Geo::STAGE;
+    static_assert(W * NS * STAGE >= W * 8 * (D + 2) * 4, "merge buffers must fit in the stages");
+
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* stages = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + W * NS * STAGE);
+    int* tbl = reinterpret_cast<int*>(bars + W * NS);
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        s_abort = 0;
+        prefetch_tensor_map(&tm_k);
+        prefetch_tensor_map(&tm_v);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < NS; ++i) mbar_init(smem_u32(&bars[warp * NS + i]), 1);
+    }
+    fence_barrier_init();
+    __syncthreads();
+
+    const int per_item = a.num_kv_heads * a.head_groups;
+    const long long units = static_cast<long long>(*a.ws_count) * per_item;
+    const int P = a.partition_size, B = a.block_size;
+    const float sl2 = a.scale_log2;
+
+    // Fragment coordinates of this lane.
+    const int g = lane >> 2, c = lane & 3;         // mma C/B fragment row group and column pair
+    const int mi = lane >> 3, rr = lane & 7;       // ldmatrix: matrix index and row within it
+    const uint32_t krow = Geo::row_off(rr + 8 * (mi & 1));
+    const uint32_t vrow = Geo::row_off(rr + 8 * (mi >> 1));
+    const uint32_t ksw = (krow >> 7) & 7, vsw = (vrow >> 7) & 7;
+    uint32_t kx[4], vx[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        kx[q4] = ((2 * q4 + (mi >> 1)) ^ ksw) << 4;
+        vx[q4] = ((2 * q4 + (mi & 1)) ^ vsw) << 4;
+    }
+
+    uint8_t* wst = stages + warp * NS * STAGE;
+    const uint32_t wst_u32 = smem_u32(wst);
+    const uint32_t wbar_u32 = smem_u32(&bars[warp * NS]);
+    uint32_t n_issued = 0, n_used = 0;   // this warp's ring position; carried across units
+
+    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+        const int item = a.ws_items[u / per_item];
+        const int r = static_cast<int>(u % per_item);
+        const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
+        const int s = item / a.max_parts, p = item - (item / a.max_parts) * a.max_parts;
+        const int ctx = clamp_context(a.context_lens[s], a.cap);
+        const int t0 = p * P;
+        const int t1 = min(t0 + P, ctx);
+        const int ntok = t1 - t0;
+        const int nparts = (ctx + P - 1) / P;
+        const int nblk = (t1 - 1) / B - t0 / B + 1;
+        const int gsub = min(8, a.group - hg * 8);
+        const int head0 = kvh * a.group + hg * 8;
+
+        __syncthreads();   // the previous unit's epilogue is done with shared memory
+        if (s_abort) break;
+
+        // block-table slice of this partition, validated once
+        int bad = 0;
+        const int32_t* trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks + t0 / B;
+        for (int i = tid; i < nblk; i += W * 32) {
+            int b = trow[i];
+            if (b < 0 || b >= a.num_blocks) {
+                b = -1;
+                bad = 1;
+            }
+            tbl[i] = b;
+        }
+        // q fragments (B operand of S^T = K Q^T): head g of the group, columns 16ks + 2c (+8)
+        uint32_t qf[KS][2];
+        if (g < gsub) {
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                static_cast<const __nv_bfloat16*>(a.q) +
+                (static_cast<size_t>(s) * a.num_heads + head0 + g) * D);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                qf[ks][0] = qrow[8 * ks + c];
+                qf[ks][1] = qrow[8 * ks + c + 4];
+            }
+        } else {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) qf[ks][0] = qf[ks][1] = 0u;
+        }
+        bad = __syncthreads_or(bad);
+        if (bad && tid == 0) flag_error(a.dev_err, PA_DEVERR_BLOCK_ID);
+
+        const int ntiles = (ntok + 15) / 16;
+        const int my_tiles = warp < ntiles ? (ntiles - warp + W - 1) / W : 0;
+
+        // Issue the bulk copies of this warp's j-th tile into the next ring stage.
+        auto issue = [&](int j) {
+            const int stage = static_cast<int>(n_issued % NS);
+            ++n_issued;
+            if (lane == 0) {
+                const int r0 = 16 * (warp + j * W);
+                const uint32_t bar = wbar_u32 + 8 * stage;
+                const uint32_t dst = wst_u32 + stage * STAGE;
+                uint32_t bytes = 0;
+#pragma unroll
+                for (int piece = 0; piece < Geo::BOXES; ++piece) {
+                    const int tok = r0 + piece * RB;
+                    if (tok < ntok && tbl[tok / B] >= 0) bytes += 2 * NH * RB * 128;
+                }
+                mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+                for (int piece = 0; piece < Geo::BOXES; ++piece) {
+                    const int tok = r0 + piece * RB;
+                    if (tok >= ntok) break;
+                    const int phys = tbl[tok / B];
+                    if (phys < 0) continue;
+                    const int y = (phys * a.num_kv_heads + kvh) * B + (tok % B);
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        tma_load_2d(dst + h * HALF + piece * Geo::BOX_STRIDE, &tm_k, bar, 64 * h, y);
+                        tma_load_2d(dst + (NH + h) * HALF + piece * Geo::BOX_STRIDE, &tm_v, bar, 64 * h, y);
+                    }
+                }
+            }
+        };
+
+        float m0 = NEG_INF, m1 = NEG_INF, l0 = 0.f, l1 = 0.f;
+        float o[KS][4];
+#pragma unroll
+        for (int i = 0; i < KS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+        const int npro = my_tiles < NS ? my_tiles : NS;
+        for (int j = 0; j < npro; ++j) issue(j);
+
+        bool failed = false;
+        for (int j = 0; j < my_tiles; ++j) {
+            const int stage = static_cast<int>(n_used % NS);
+            const uint32_t parity = (n_used / NS) & 1u;
+            const bool arrived = mbar_wait_bounded(wbar_u32 + 8 * stage, parity, WAIT_LIMIT_NS);
+            if (!__all_sync(FULL_MASK, arrived)) {   // keep the warp together on a timeout
+                failed = true;
+                break;
+            }
+            ++n_used;
+            const uint32_t st = wst_u32 + stage * STAGE;
+            const int r0 = 16 * (warp + j * W);
+
+            // tokens of this tile that take part: inside the partition and in a valid block
+            unsigned mask = 0xffffu;
+            if (r0 + 16 > ntok || bad) {
+                const int tok = r0 + (lane & 15);
+                const bool ok = tok < ntok && tbl[tok / B] >= 0;
+                mask = __ballot_sync(FULL_MASK, ok) & 0xffffu;
+                // value rows of excluded tokens may hold anything (NaN included): zero them
+                uint8_t* stp = wst + stage * STAGE;
+                for (int idx = lane; idx < 16 * NH * 8; idx += 32) {
+                    const int row = idx / (NH * 8), rem = idx % (NH * 8);
+                    if (!((mask >> row) & 1u))
+                        *reinterpret_cast<uint4*>(stp + (NH + rem / 8) * HALF + Geo::row_off(row) +
+                                                  (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+
+            // S^T (16 tokens x 8 heads) = K (16 x D) . Q^T (D x 8)
+            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4(st + (ks / 4) * HALF + krow + kx[ks % 4], a0, a1, a2, a3);
+                mma_bf16_16816(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+            }
+            // logits in the log2 domain; rows g and g+8 are tokens, columns 2c, 2c+1 heads
+            float x0 = sc[0] * sl2, x1 = sc[1] * sl2, x2 = sc[2] * sl2, x3 = sc[3] * sl2;
+            if (mask != 0xffffu) {
+                if (!((mask >> g) & 1u)) x0 = x1 = NEG_INF;
+                if (!((mask >> (g + 8)) & 1u)) x2 = x3 = NEG_INF;
+            }
+            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
+            }
+            const bool up0 = mx0 > m0 + RESCALE_THRESHOLD, up1 = mx1 > m1 + RESCALE_THRESHOLD;
+            if (__any_sync(FULL_MASK, up0 || up1)) {
+                const float al0 = up0 ? exp2_approx(m0 - mx0) : 1.f;
+                const float al1 = up1 ? exp2_approx(m1 - mx1) : 1.f;
+                if (up0) m0 = mx0;
+                if (up1) m1 = mx1;
+                l0 *= al0;
+                l1 *= al1;
+#pragma unroll
+                for (int i = 0; i < KS; ++i) {
+                    o[i][0] *= al0;
+                    o[i][1] *= al1;
+                    o[i][2] *= al0;
+                    o[i][3] *= al1;
+                }
+            }
+            const float b0 = m0 == NEG_INF ? 0.f : m0, b1 = m1 == NEG_INF ? 0.f : m1;
+            const float p0 = exp2_approx(x0 - b0), p1 = exp2_approx(x1 - b1);
+            const float p2 = exp2_approx(x2 - b0), p3 = exp2_approx(x3 - b1);
+            l0 += p0 + p2;
+            l1 += p1 + p3;
+            // weights as a bf16 pair hi + lo (about 16 significant bits), transposed
+            // into the B operand of O^T (D x 8) += V^T (D x 16) . P^T (16 x 8)
+            const uint32_t h01 = pack_bf16(p0, p1), h23 = pack_bf16(p2, p3);
+            const uint32_t q01 = pack_bf16(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
+            const uint32_t q23 = pack_bf16(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
+            const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+            const uint32_t bl0 = movmatrix_trans(q01), bl1 = movmatrix_trans(q23);
+#pragma unroll
+            for (int i = 0; i < KS; ++i) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4_trans(st + (NH + i / 4) * HALF + vrow + vx[i % 4], a0, a1, a2, a3);
+                mma_bf16_16816(o[i], a0, a1, a2, a3, bh0, bh1);
+                mma_bf16_16816(o[i], a0, a1, a2, a3, bl0, bl1);
+            }
+            __syncwarp();
+            if (j + NS < my_tiles) issue(j + NS);
+        }
+        if (failed) {
+            if (lane == 0) {
+                flag_error(a.dev_err, PA_DEVERR_TIMEOUT);
+                s_abort = 1;
+            }
+            // wait, again bounded, for this warp's copies still in flight
+            while (n_used < n_issued) {
+                const int stage = static_cast<int>(n_used % NS);
+                mbar_wait_bounded(wbar_u32 + 8 * stage, (n_used / NS) & 1u, DRAIN_LIMIT_NS);
+                ++n_used;
+            }
+        }
+
+        // row sums over the 8 lanes that share a head pair
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l0 += __shfl_xor_sync(FULL_MASK, l0, off);
+            l1 += __shfl_xor_sync(FULL_MASK, l1, off);
+        }
+        __syncthreads();   // every warp is done with its stages
+        float* mm = reinterpret_cast<float*>(stages);
+        float* ml = mm + W * 8;
+        float* mo = ml + W * 8;
+        if (g == 0) {
+            mm[warp * 8 + 2 * c] = m0;
+            mm[warp * 8 + 2 * c + 1] = m1;
+            ml[warp * 8 + 2 * c] = l0;
+            ml[warp * 8 + 2 * c + 1] = l1;
+        }
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+            mo[(warp * 8 + 2 * c) * D + 16 * i + g] = o[i][0];
+            mo[(warp * 8 + 2 * c + 1) * D + 16 * i + g] = o[i][1];
+            mo[(warp * 8 + 2 * c) * D + 16 * i + 8 + g] = o[i][2];
+            mo[(warp * 8 + 2 * c + 1) * D + 16 * i + 8 + g] = o[i][3];
+        }
+        __syncthreads();
+        combine_store<W, D>(a, mm, ml, mo, s, p, nparts, head0, gsub);
+        fence_proxy_async_smem();   // these generic accesses precede the next unit's bulk copies
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2b. attend, fp32: CUDA cores, one warp per token, lanes split the head dim
+// ---------------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(128) attend_f32_kernel(const DecodeArgs a) {
+    constexpr int W = 4, J = D / 32;
+    __shared__ float mm[W * 8], ml[W * 8];
+    __shared__ float mo[W * 8 * D];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int per_item = a.num_kv_heads * a.head_groups;
+    const long long units = static_cast<long long>(*a.ws_count) * per_item;
+    const int P = a.partition_size, B = a.block_size;
+    const float* kc = static_cast<const float*>(a.k_cache);
+    const float* vc = static_cast<const float*>(a.v_cache);
+    const float* qp = static_cast<const float*>(a.q);
+
+    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+        const int item = a.ws_items[u / per_item];
+        const int r = static_cast<int>(u % per_item);
+        const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
+        const int s = item / a.max_parts, p = item - (item / a.max_parts) * a.max_parts;
+        const int ctx = clamp_context(a.context_lens[s], a.cap);
+        const int t0 = p * P, t1 = min(t0 + P, ctx);
+        const int nparts = (ctx + P - 1) / P;
+        const int gsub = min(8, a.group - hg * 8);
+        const int head0 = kvh * a.group + hg * 8;
+
+        float qv[8][J], acc[8][J], m[8], l[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            m[n] = NEG_INF;
+            l[n] = 0.f;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                acc[n][j] = 0.f;
+                qv[n][j] = n < gsub ? qp[(static_cast<size_t>(s) * a.num_heads + head0 + n) * D + lane + 32 * j]
+                                    : 0.f;
+            }
+        }
+        for (int t = t0 + warp; t < t1; t += W) {
+            const int phys = a.block_tables[static_cast<size_t>(s) * a.max_blocks + t / B];
+            if (phys < 0 || phys >= a.num_blocks) {
+                if (lane == 0) flag_error(a.dev_err, PA_DEVERR_BLOCK_ID);
+                continue;
+            }
+            const size_t rowi = ((static_cast<size_t>(phys) * a.num_kv_heads + kvh) * B + t % B) * D;
+            float kv[J], vv[J];
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                kv[j] = kc[rowi + lane + 32 * j];
+                vv[j] = vc[rowi + lane + 32 * j];
+            }
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                if (n >= gsub) break;
+                float dot = 0.f;
+#pragma unroll
+                for (int j = 0; j < J; ++j) dot = fmaf(qv[n][j], kv[j], dot);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(FULL_MASK, dot, off);
+                const float x = dot * a.scale_log2;
+                const float mn = fmaxf(m[n], x);
+                const float al = exp2_approx(m[n] - mn);
+                const float pw = exp2_approx(x - mn);
+                l[n] = l[n] * al + pw;
+#pragma unroll
+                for (int j = 0; j < J; ++j) acc[n][j] = fmaf(pw, vv[j], acc[n][j] * al);
+                m[n] = mn;
+            }
+        }
+        __syncthreads();   // the previous unit's epilogue is done with the merge buffers
+        if (lane == 0) {
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                mm[warp * 8 + n] = m[n];
+                ml[warp * 8 + n] = l[n];
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+#pragma unroll
+            for (int j = 0; j < J; ++j) mo[(warp * 8 + n) * D + lane + 32 * j] = acc[n][j];
+        __syncthreads();
+        combine_store<W, D>(a, mm, ml, mo, s, p, nparts, head0, gsub);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. reduce: merge the partitions of one (seq, head), in partition order
+// ---------------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
+    constexpr int J = D / 32;
+    __shared__ float red[4];
+    __shared__ float so[4][D];
+    __shared__ float sl[4];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int s = blockIdx.x / a.num_heads, head = blockIdx.x - (blockIdx.x / a.num_heads) * a.num_heads;
+    const int ctx = clamp_context(a.context_lens[s], a.cap);
+    const int P = a.partition_size;
+    const int nparts = (ctx + P - 1) / P;
+    if (nparts == 1) return;   // written directly by the attend kernel
+    const size_t row = static_cast<size_t>(s) * a.num_heads + head;
+    if (nparts == 0) {
+        for (int d = tid; d < D; d += 128) {
+            if (a.out_f32)
+                static_cast<float*>(a.out)[row * D + d] = 0.f;
+            else
+                static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(0.f);
+        }
+        return;
+    }
+    const float2* mlp = a.ws_ml + row * a.max_parts;
+    const float* accp = a.ws_acc + row * a.max_parts * D;
+    float M = NEG_INF;
+    for (int p = tid; p < nparts; p += 128) M = fmaxf(M, mlp[p].x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    float L = 0.f, o[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) o[j] = 0.f;
+    if (M != NEG_INF) {
+        for (int p = warp; p < nparts; p += 4) {
+            const float2 v = mlp[p];
+            const float e = exp2_approx(v.x - M);
+            L += e * v.y;
+#pragma unroll
+            for (int j = 0; j < J; ++j) o[j] = fmaf(e, accp[static_cast<size_t>(p) * D + lane + 32 * j], o[j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < J; ++j) so[warp][lane + 32 * j] = o[j];
+    if (lane == 0) sl[warp] = L;
+    __syncthreads();
+    const float Lt = (sl[0] + sl[1]) + (sl[2] + sl[3]);
+    for (int d = tid; d < D; d += 128) {
+        const float O = (so[0][d] + so[1][d]) + (so[2][d] + so[3][d]);
+        const float v = Lt > 0.f ? O / Lt : 0.f;
+        if (a.out_f32)
+            static_cast<float*>(a.out)[row * D + d] = v;
+        else
+            static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(v);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+constexpr int ATTEND_WARPS = 4;
+constexpr int ATTEND_STAGES = 3;
+
+inline size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+struct WsLayout {
+    size_t items, ml, acc, total;
+};
+
+inline WsLayout ws_layout(int S, int Hq, int D, int max_parts) {
+    WsLayout L;
+    size_t off = 256;   // header: the work-item count
+    L.items = off;
+    off += round_up(static_cast<size_t>(S) * max_parts * sizeof(int), 256);
+    if (max_parts > 1) {
+        L.ml = off;
+        off += round_up(static_cast<size_t>(S) * Hq * max_parts * sizeof(float2), 256);
+        L.acc = off;
+        off += round_up(static_cast<size_t>(S) * Hq * max_parts * D * sizeof(float), 256);
+    } else {
+        L.ml = L.acc = 0;
+    }
+    L.total = off;
+    return L;
+}
+
+inline int parts_for(int cap, int P) {
+    const int n = (cap + P - 1) / P;
+    return n < 1 ? 1 : n;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (f) return f;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || ptr == nullptr)
+        return nullptr;
+    f = reinterpret_cast<EncodeTiledFn>(ptr);
+    fn.store(f, std::memory_order_release);
+    return f;
+}
+
+// Tensor map over one bf16 pool viewed as rows of head_dim elements
+// (row = (block * Hkv + kv_head) * B + slot), boxes of 64 columns x rb rows.
+inline bool encode_pool_map(CUtensorMap* m, const void* pool, int num_blocks, int Hkv, int B, int D,
+                            int rb) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D),
+                                static_cast<cuuint64_t>(num_blocks) * Hkv * B};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(rb)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int RB>
+int launch_attend_bf16(const DecodeArgs& a, cudaStream_t st, long long unit_bound) {
+    using Geo = TileGeom<D, RB>;
+    constexpr int W = ATTEND_WARPS, NS = ATTEND_STAGES;
+    static KernelSlot slot;
+    CUtensorMap tk, tv;
+    if (!encode_pool_map(&tk, a.k_cache, a.num_blocks, a.num_kv_heads, a.block_size, D, RB) ||
+        !encode_pool_map(&tv, a.v_cache, a.num_blocks, a.num_kv_heads, a.block_size, D, RB))
+        return PA_ERR_CUDA;
+    const int tbl_entries = a.partition_size / a.block_size;
+    const int smem = 1024 + W * NS * Geo::STAGE + W * NS * 8 + tbl_entries * 4;
+    auto kern = attend_bf16_kernel<D, RB, W, NS>;
+    const int per_sm = prepare_kernel(slot, reinterpret_cast<const void*>(kern), W * 32, smem);
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (per_sm <= 0 || sms <= 0) return PA_ERR_CUDA;
+    const long long cap_ctas = static_cast<long long>(per_sm) * sms;
+    const int grid = static_cast<int>(unit_bound < cap_ctas ? unit_bound : cap_ctas);
+    if (grid <= 0) return PA_OK;
+    kern<<<grid, W * 32, smem, st>>>(tk, tv, a);
+    return launch_status();
+}
+
+template <int D>
+int launch_attend_f32(const DecodeArgs& a, cudaStream_t st, long long unit_bound) {
+    static KernelSlot slot;
+    auto kern = attend_f32_kernel<D>;
+    const int per_sm = prepare_kernel(slot, reinterpret_cast<const void*>(kern), 128, 0);
+    const int sms = current_sm_count();
+    if (per_sm <= 0 || sms <= 0) return PA_ERR_CUDA;
+    const long long cap_ctas = static_cast<long long>(per_sm) * sms;
+    const int grid = static_cast<int>(unit_bound < cap_ctas ? unit_bound : cap_ctas);
+    if (grid <= 0) return PA_OK;
+    kern<<<grid, 128, 0, st>>>(a);
+    return launch_status();
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                            int max_context_len, int partition_size) {
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 || partition_size <= 0)
+        return 0;
+    return ws_layout(num_seqs, num_heads, head_dim, parts_for(max_context_len, partition_size)).total;
+}
+
+extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, int num_seqs, int num_heads,
+                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                int max_blocks_per_seq, int max_context_len, float scale,
+                                int partition_size, void* workspace, size_t workspace_bytes,
+                                pa_dtype dtype, int32_t* dev_err, pa_stream stream, int phases) {
+    // ---- host-side validation: nothing is launched unless everything is sane
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !valid_dtype(out_dtype)) return PA_ERR_INVALID_ARG;
+    if (out_dtype != PA_F32 && out_dtype != dtype) return PA_ERR_UNSUPPORTED;
+    if (!(head_dim == 64 || head_dim == 128)) return PA_ERR_UNSUPPORTED;
+    if (!(block_size == 4 || block_size == 8 || block_size == 16 || block_size == 32))
+        return PA_ERR_UNSUPPORTED;
+    if (partition_size < 32 || partition_size > 8192 || partition_size % 32 != 0 ||
+        partition_size % block_size != 0)
+        return PA_ERR_UNSUPPORTED;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if ((phases & ~PA_PHASE_ALL) != 0 || phases == 0) return PA_ERR_INVALID_ARG;
+    if (static_cast<long long>(num_blocks) * num_kv_heads * block_size > INT_MAX)
+        return PA_ERR_UNSUPPORTED;   // bulk-copy row coordinates are 32-bit
+    if (static_cast<long long>(max_blocks_per_seq) * block_size > INT_MAX) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+
+    long long cap = static_cast<long long>(max_blocks_per_seq) * block_size;
+    if (max_context_len > 0 && max_context_len < cap) cap = max_context_len;
+    const int max_parts = parts_for(static_cast<int>(cap), partition_size);
+    if (static_cast<long long>(num_seqs) * max_parts > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, max_parts);
+    if (!workspace || !aligned_to(workspace, 256)) return PA_ERR_INVALID_ARG;
+    if (workspace_bytes < L.total) return PA_ERR_WORKSPACE;
+    if (!context_lens || !aligned_to(context_lens, 4)) return PA_ERR_INVALID_ARG;
+    if (phases & (PA_PHASE_ATTEND | PA_PHASE_REDUCE)) {
+        if (!out || !aligned_to(out, 16)) return PA_ERR_INVALID_ARG;
+    }
+    if (phases & PA_PHASE_ATTEND) {
+        if (!q || !k_cache || !v_cache || !block_tables) return PA_ERR_INVALID_ARG;
+        if (!aligned_to(q, 16) || !aligned_to(k_cache, 16) || !aligned_to(v_cache, 16) ||
+            !aligned_to(block_tables, 4))
+            return PA_ERR_INVALID_ARG;
+    }
+
+    DecodeArgs a;
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.dev_err = dev_err;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.ws_count = reinterpret_cast<int*>(ws);
+    a.ws_items = reinterpret_cast<int*>(ws + L.items);
+    a.ws_ml = max_parts > 1 ? reinterpret_cast<float2*>(ws + L.ml) : nullptr;
+    a.ws_acc = max_parts > 1 ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.head_dim = head_dim;
+    a.block_size = block_size;
+    a.num_blocks = num_blocks;
+    a.max_blocks = max_blocks_per_seq;
+    a.cap = static_cast<int>(cap);
+    a.partition_size = partition_size;
+    a.max_parts = max_parts;
+    a.group = num_heads / num_kv_heads;
+    a.head_groups = (a.group + 7) / 8;
+    a.scale_log2 = scale * LOG2E;
+    a.out_f32 = out_dtype == PA_F32;
+    const cudaStream_t st = as_stream(stream);
+
+    if (phases & PA_PHASE_PLAN) {
+        plan_kernel<<<1, PLAN_THREADS, 0, st>>>(a);
+        if (launch_status() != PA_OK) return PA_ERR_CUDA;
+    }
+    if (phases & PA_PHASE_ATTEND) {
+        const long long unit_bound =
+            static_cast<long long>(num_seqs) * max_parts * num_kv_heads * a.head_groups;
+        int rc;
+        if (dtype == PA_BF16) {
+            const int rb = block_size < 16 ? block_size : 16;
+            if (head_dim == 128)
+                rc = rb == 16 ? launch_attend_bf16<128, 16>(a, st, unit_bound)
+                     : rb == 8 ? launch_attend_bf16<128, 8>(a, st, unit_bound)
+                               : launch_attend_bf16<128, 4>(a, st, unit_bound);
+            else
+                rc = rb == 16 ? launch_attend_bf16<64, 16>(a, st, unit_bound)
+                     : rb == 8 ? launch_attend_bf16<64, 8>(a, st, unit_bound)
+                               : launch_attend_bf16<64, 4>(a, st, unit_bound);
+        } else {
+            rc = head_dim == 128 ? launch_attend_f32<128>(a, st, unit_bound)
+                                 : launch_attend_f32<64>(a, st, unit_bound);
+        }
+        if (rc != PA_OK) return rc;
+    }
+    if (phases & PA_PHASE_REDUCE) {
+        const long long rows = static_cast<long long>(num_seqs) * num_heads;
+        if (rows > INT_MAX) return PA_ERR_UNSUPPORTED;
+        if (head_dim == 128)
+            reduce_kernel<128><<<static_cast<int>(rows), 128, 0, st>>>(a);
+        else
+            reduce_kernel<64><<<static_cast<int>(rows), 128, 0, st>>>(a);
+        if (launch_status() != PA_OK) return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
+extern "C" int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                         const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                         int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                         int partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                         int32_t* dev_err, pa_stream stream) {
+    return pa_decode_phases(out, out_dtype, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                            num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                            max_blocks_per_seq, max_context_len, scale, partition_size, workspace,
+                            workspace_bytes, dtype, dev_err, stream, PA_PHASE_ALL);
+}

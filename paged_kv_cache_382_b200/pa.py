@@ -1,0 +1,184 @@
+"""ctypes binding of libpa.so: argument marshalling only.
+
+Every function checks the torch tensors it is given (device, dtype,
+contiguity), passes raw device pointers and the current CUDA stream to the C
+ABI declared in ``include/pa.h``, and raises ``PagedAttentionError`` on a
+non-zero status.  All arithmetic happens in the library's CUDA kernels; there
+is no CPU fallback -- importing this module raises ImportError when libpa.so
+has not been built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
+
+PA_F32, PA_BF16 = 0, 1
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, 1, 2, 3, 4
+DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_CONTEXT, DEVERR_COPY, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+PHASE_PLAN, PHASE_ATTEND, PHASE_REDUCE, PHASE_ALL = 0x1, 0x2, 0x4, 0x7
+
+_vp, _i, _i32p, _i64p, _sz, _f = (ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.c_size_t, ctypes.c_float)
+
+_DECODE_ARGS = [_vp, _i, _vp, _vp, _vp, _i32p, _i32p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                _vp, _sz, _i, _i32p, _vp]
+
+SIGNATURES = {
+    "pa_reshape_and_cache": (_i, [_vp, _vp, _vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _i32p, _vp]),
+    "pa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "pa_decode": (_i, _DECODE_ARGS),
+    "pa_decode_phases": (_i, _DECODE_ARGS + [_i]),
+    "pa_copy_blocks": (_i, [_vp, _vp, _i64p, _i, _sz, _i, _i32p, _vp]),
+    "pa_status_string": (ctypes.c_char_p, [_i]),
+    "pa_version": (_i, []),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built: run `python -m paged_kv_cache_382_b200.build` "
+            "(needs nvcc); this package has no CPU fallback")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (restype, argtypes) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = restype
+        fn.argtypes = argtypes
+    return lib
+
+
+lib = _load()
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {lib.pa_status_string(status).decode()}")
+        self.status = status
+
+
+def _check(status: int, what: str) -> None:
+    if status != PA_OK:
+        raise PagedAttentionError(what, status)
+
+
+def dtype_code(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return PA_F32
+    if dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"unsupported dtype {dtype}; the kernels take float32 or bfloat16")
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _opt_err(dev_err: Optional[torch.Tensor]) -> Optional[int]:
+    if dev_err is None:
+        return None
+    return _dev(dev_err, "dev_err", torch.int32)
+
+
+def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor,
+                      v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                      dev_err: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Write key/value [T][Hkv][d] into the pools [NB][Hkv][B][d] at slot_mapping (int64 [T])."""
+    NB, Hkv, B, d = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache must have the same shape")
+    T = key.shape[0]
+    if tuple(key.shape) != (T, Hkv, d) or tuple(value.shape) != (T, Hkv, d):
+        raise ValueError("key/value must be [num_tokens][num_kv_heads][head_dim]")
+    if tuple(slot_mapping.shape) != (T,):
+        raise ValueError("slot_mapping must be [num_tokens]")
+    dt = k_cache.dtype
+    rc = lib.pa_reshape_and_cache(
+        _dev(key, "key", dt), _dev(value, "value", dt), _dev(k_cache, "k_cache", dt),
+        _dev(v_cache, "v_cache", dt), _dev(slot_mapping, "slot_mapping", torch.int64), T, Hkv, d, B,
+        NB, dtype_code(dt), _opt_err(dev_err), _stream_handle(stream))
+    _check(rc, "pa_reshape_and_cache")
+
+
+def decode_workspace_bytes(num_seqs: int, num_heads: int, head_dim: int, max_context_len: int,
+                           partition_size: int = 512) -> int:
+    n = lib.pa_decode_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size)
+    if n == 0:
+        raise ValueError("invalid arguments for pa_decode_workspace_bytes")
+    return int(n)
+
+
+def decode_capacity(block_tables: torch.Tensor, block_size: int, max_context_len: int = 0) -> int:
+    """The context bound the library uses: max_context_len, or max_blocks * block_size if 0."""
+    cap = block_tables.shape[1] * block_size
+    return cap if max_context_len <= 0 else min(cap, max_context_len)
+
+
+def alloc_workspace(num_seqs: int, num_heads: int, head_dim: int, capacity: int,
+                    partition_size: int = 512, device=None) -> torch.Tensor:
+    n = decode_workspace_bytes(num_seqs, num_heads, head_dim, capacity, partition_size)
+    return torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, *,
+           max_context_len: int = 0, partition_size: int = 512,
+           workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+           stream: Optional[torch.cuda.Stream] = None, phases: int = PHASE_ALL) -> torch.Tensor:
+    """Paged decode attention; writes and returns ``out`` [S][Hq][d]."""
+    NB, Hkv, B, d = k_cache.shape
+    S, Hq, dq = q.shape
+    if dq != d or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q, k_cache and v_cache disagree on head_dim / shape")
+    if tuple(out.shape) != (S, Hq, d):
+        raise ValueError("out must be [num_seqs][num_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [num_seqs][max_blocks] and context_lens [num_seqs]")
+    dt = k_cache.dtype
+    if workspace is None:
+        cap = decode_capacity(block_tables, B, max_context_len)
+        workspace = alloc_workspace(S, Hq, d, cap, partition_size, q.device)
+    rc = lib.pa_decode_phases(
+        _dev(out, "out"), dtype_code(out.dtype), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt),
+        _dev(v_cache, "v_cache", dt), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), S, Hq, Hkv, d, B, NB,
+        block_tables.shape[1], max_context_len, float(scale), partition_size,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), dtype_code(dt),
+        _opt_err(dev_err), _stream_handle(stream), phases)
+    _check(rc, "pa_decode")
+    return out
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: torch.Tensor,
+                dev_err: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Copy whole blocks src -> dst (int64 [n][2] on the device) in both pools."""
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or v_cache.dtype != k_cache.dtype:
+        raise ValueError("k_cache and v_cache must match")
+    n = src_dst_pairs.shape[0]
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [num_pairs][2]")
+    block_bytes = k_cache[0].numel() * k_cache.element_size()
+    rc = lib.pa_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                            _dev(src_dst_pairs, "src_dst_pairs", torch.int64), n, block_bytes,
+                            k_cache.shape[0], _opt_err(dev_err), _stream_handle(stream))
+    _check(rc, "pa_copy_blocks")

@@ -1,0 +1,397 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bars, from the decode-attention target: scatter and block copies bit-exact;
+decode max |err| <= 1e-5 for fp32 inputs and <= 2e-3 for bf16 inputs with fp32
+accumulation (fp32 output); a bf16 output may differ by a further half bf16 ulp
+of the exact value, the rounding of the output itself.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_382_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 2e-3
+
+
+@pytest.fixture(scope="module")
+def pa():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    from paged_kv_cache_382_b200 import build
+
+    build.build()
+    from paged_kv_cache_382_b200 import pa as binding
+
+    return binding
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+class SparsePool:
+    """Some blocks of a pool, indexed by physical id like the full array.
+
+    Lets the oracle run on the blocks one sequence touches without copying a
+    multi-gigabyte pool to the host."""
+
+    def __init__(self, blocks, shape):
+        self.blocks = blocks
+        self.shape = shape
+
+    @classmethod
+    def fetch(cls, pool: torch.Tensor, ids, as_float=True):
+        ids = sorted(set(int(i) for i in ids))
+        idx = torch.tensor(ids, dtype=torch.long, device=pool.device)
+        rows = pool.index_select(0, idx)
+        rows = rows.to("cpu", torch.float64).numpy() if as_float else raw_bits(rows)
+        return cls({b: rows[i].copy() for i, b in enumerate(ids)}, tuple(pool.shape))
+
+    def copy(self):
+        return SparsePool({k: v.copy() for k, v in self.blocks.items()}, self.shape)
+
+    def __getitem__(self, idx):
+        if isinstance(idx, tuple):
+            return self.blocks[int(idx[0])][idx[1:]]
+        return self.blocks[int(idx)]
+
+    def __setitem__(self, idx, val):
+        if isinstance(idx, tuple):
+            self.blocks[int(idx[0])][idx[1:]] = val
+        else:
+            self.blocks[int(idx)] = np.array(val, copy=True)
+
+
+def raw_bits(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu().contiguous()
+    return t.view(torch.int16 if t.element_size() == 2 else torch.int32).numpy()
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def to_device(step: W.DecodeStep, device="cuda") -> W.DecodeStep:
+    for name in ("q", "k_cache", "v_cache", "new_key", "new_value"):
+        setattr(step, name, getattr(step, name).to(device))
+    return step
+
+
+def run_gpu(pa, step, out_dtype=torch.float32, partition_size=None, max_context_len=0,
+            keep_pre=False, tables=None, slots=None, pairs=None, ctx=None):
+    dev = "cuda"
+    pre = (step.k_cache.clone(), step.v_cache.clone()) if keep_pre else None
+    kc, vc = step.k_cache.clone(), step.v_cache.clone()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    pairs = step.copy_pairs if pairs is None else pairs
+    if len(pairs):
+        pa.copy_blocks(kc, vc, torch.from_numpy(np.ascontiguousarray(pairs)).to(dev), dev_err=err)
+    slots = step.slot_mapping if slots is None else slots
+    if len(slots):
+        pa.reshape_and_cache(step.new_key, step.new_value, kc, vc, torch.from_numpy(slots).to(dev),
+                             dev_err=err)
+    tables = step.block_tables if tables is None else tables
+    ctx = step.context_lens if ctx is None else ctx
+    out = torch.empty(step.num_seqs, step.num_heads, step.head_dim, dtype=out_dtype, device=dev)
+    pa.decode(out, step.q, kc, vc, torch.from_numpy(np.ascontiguousarray(tables, dtype=np.int32)).to(dev),
+              torch.from_numpy(np.ascontiguousarray(ctx, dtype=np.int32)).to(dev), step.scale,
+              partition_size=partition_size or step.partition_size, max_context_len=max_context_len,
+              dev_err=err)
+    torch.cuda.synchronize()
+    return out, kc, vc, int(err.item()), pre
+
+
+def oracle_outputs(step, seqs, pre_k, pre_v):
+    """Oracle output rows for the given sequences, from the pool as it was before
+    this step's copies and writes (pre_k / pre_v on the device)."""
+    res = {}
+    B = step.block_size
+    for s in seqs:
+        c = int(step.context_lens[s])
+        table = step.block_tables[s]
+        blocks = [int(b) for b in table[: -(-c // B)]]
+        pairs = [(int(a), int(b)) for a, b in step.copy_pairs if int(b) in blocks]
+        need = set(blocks) | {a for a, _ in pairs}
+        if not need:
+            res[s] = np.zeros((step.num_heads, step.head_dim))
+            continue
+        kp = SparsePool.fetch(pre_k, need)
+        vp = SparsePool.fetch(pre_v, need)
+        kp, vp = oracle.copy_blocks(kp, vp, pairs)
+        # this sequence's token of the step is row s of the step's writes
+        mine = [t for t in range(len(step.slot_mapping)) if t == s and step.slot_mapping[t] >= 0]
+        if mine:
+            t = mine[0]
+            kp, vp = oracle.reshape_and_cache(f64(step.new_key[t:t + 1]), f64(step.new_value[t:t + 1]),
+                                              kp, vp, step.slot_mapping[t:t + 1])
+        res[s] = oracle.decode_attention(f64(step.q[s:s + 1]), kp, vp, table[None], np.array([c]),
+                                         step.scale)[0]
+    return res
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, 2.0 ** (e - 8), 0.0)
+
+
+def assert_close(got, ref, dtype_in, out_dtype, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    tol = TOL_F32 if dtype_in == torch.float32 else TOL_BF16
+    bound = tol + (bf16_half_ulp(ref) if out_dtype == torch.bfloat16 else 0.0)
+    worst = float((err - bound).max())
+    assert worst <= 0.0, f"{what}: max |err| {float(err.max()):.3e} exceeds the bound by {worst:.3e}"
+    return float(err.max())
+
+
+# ---------------------------------------------------------------------------
+# small cases: every output row against the oracle
+# ---------------------------------------------------------------------------
+
+def full_oracle(step):
+    kc, vc = f64(step.k_cache), f64(step.v_cache)
+    kc, vc = oracle.copy_blocks(kc, vc, step.copy_pairs)
+    kc, vc = oracle.reshape_and_cache(f64(step.new_key), f64(step.new_value), kc, vc, step.slot_mapping)
+    return oracle.decode_attention(f64(step.q), kc, vc, step.block_tables, step.context_lens, step.scale)
+
+
+@pytest.mark.parametrize("block_size", [16, 4])
+@pytest.mark.parametrize("partition_size", [512, 32])
+def test_tiny_fp32(pa, block_size, partition_size):
+    step = to_device(W.tiny(block_size=block_size, poison=True))
+    out, *_ = run_gpu(pa, step, partition_size=partition_size)
+    err = assert_close(f64(out), full_oracle(step), torch.float32, torch.float32, "tiny fp32")
+    assert err < TOL_F32
+
+
+SMALL_BF16 = [
+    # (ctx lens, Hq, Hkv, d, B, P)
+    ([7, 16, 33, 100], 4, 4, 64, 16, 512),
+    ([7, 16, 33, 100], 4, 4, 64, 4, 32),
+    ([1, 2, 15, 16, 17, 31, 33, 257], 8, 2, 128, 16, 64),
+    ([0, 5, 300, 1000], 32, 8, 128, 16, 512),
+    ([0, 5, 300, 1000], 32, 8, 128, 8, 128),
+    ([1, 40, 613, 1024, 1025], 64, 8, 128, 32, 512),
+    ([129, 3, 77], 16, 1, 128, 16, 32),
+    ([50, 513, 9], 6, 2, 64, 8, 64),
+    ([700, 1], 12, 1, 64, 4, 96),
+    ([2049, 64], 8, 8, 128, 32, 8192),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_BF16, ids=lambda c: f"ctx{len(c[0])}_h{c[1]}x{c[2]}_d{c[3]}_b{c[4]}_p{c[5]}")
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32out", "bf16out"])
+def test_small_bf16(pa, case, out_dtype):
+    ctx, Hq, Hkv, d, B, P = case
+    step = to_device(W.independent("small", ctx, dtype=torch.bfloat16, num_heads=Hq, num_kv_heads=Hkv,
+                                   head_dim=d, block_size=B, seed=len(ctx) + Hq + B, poison=True,
+                                   partition_size=P))
+    out, _, _, err, _ = run_gpu(pa, step, out_dtype=out_dtype)
+    assert err == 0
+    assert_close(f64(out), full_oracle(step), torch.bfloat16, out_dtype, str(case))
+
+
+def test_many_sequences_plan_chunks(pa):
+    """More sequences than the plan kernel's 1024 threads, lengths 0..40."""
+    rng = np.random.default_rng(11)
+    ctx = rng.integers(0, 41, size=3000)
+    step = to_device(W.independent("many", ctx, dtype=torch.bfloat16, num_heads=8, num_kv_heads=2,
+                                   head_dim=64, block_size=8, seed=3, partition_size=32))
+    out, _, _, err, _ = run_gpu(pa, step)
+    assert err == 0
+    ref = full_oracle(step)
+    assert_close(f64(out), ref, torch.bfloat16, torch.float32, "many sequences")
+
+
+# ---------------------------------------------------------------------------
+# the cache writes: bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_reshape_and_cache_bit_exact_small(pa, dtype):
+    step = to_device(W.independent("w", [1, 4, 5, 0, 33, 16, 17], dtype=dtype, num_heads=4, num_kv_heads=4,
+                                   head_dim=64 if dtype == torch.float32 else 128, block_size=4, seed=5))
+    kc, vc = step.k_cache.clone(), step.v_cache.clone()
+    pa.reshape_and_cache(step.new_key, step.new_value, kc, vc, torch.from_numpy(step.slot_mapping).cuda())
+    torch.cuda.synchronize()
+    ek, ev = oracle.reshape_and_cache(raw_bits(step.new_key), raw_bits(step.new_value),
+                                      raw_bits(step.k_cache), raw_bits(step.v_cache), step.slot_mapping)
+    assert np.array_equal(raw_bits(kc), ek) and np.array_equal(raw_bits(vc), ev)
+
+
+def test_copy_blocks_bit_exact_small(pa):
+    step = to_device(W.shared_prefix(prompt_len=520, suffix_max=0, prompts=2, samples=4))
+    assert len(step.copy_pairs) == 2 * 3
+    kc, vc = step.k_cache.clone(), step.v_cache.clone()
+    pa.copy_blocks(kc, vc, torch.from_numpy(step.copy_pairs).cuda())
+    torch.cuda.synchronize()
+    ek, ev = oracle.copy_blocks(raw_bits(step.k_cache), raw_bits(step.v_cache), step.copy_pairs)
+    assert np.array_equal(raw_bits(kc), ek) and np.array_equal(raw_bits(vc), ev)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the benchmark times
+# ---------------------------------------------------------------------------
+
+FULL = {
+    "llama7b": lambda: W.llama7b(device="cuda"),
+    "gqa": lambda: W.gqa(device="cuda"),
+    "shared_prefix_p512": lambda: W.shared_prefix(prompt_len=512, suffix_max=512, device="cuda"),
+    "shared_prefix_p520_cow": lambda: W.shared_prefix(prompt_len=520, suffix_max=0, device="cuda"),
+    "long_context_b8": lambda: W.long_context(block_size=8, device="cuda"),
+    "long_context_b16": lambda: W.long_context(block_size=16, device="cuda"),
+    "long_context_b32": lambda: W.long_context(block_size=32, device="cuda"),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size(pa, name):
+    step = FULL[name]()
+    out, kc, vc, err, pre = run_gpu(pa, step, keep_pre=True)
+    assert err == 0
+    assert torch.isfinite(out).all()
+    pre_k, pre_v = pre
+    # cache writes: every touched block bit-exact, every other block untouched
+    touched = sorted({int(s) // step.block_size for s in step.slot_mapping if s >= 0}
+                     | {int(b) for _, b in step.copy_pairs})
+    srcs = {int(a) for a, _ in step.copy_pairs}
+    kp = SparsePool.fetch(pre_k, set(touched) | srcs, as_float=False)
+    vp = SparsePool.fetch(pre_v, set(touched) | srcs, as_float=False)
+    kp, vp = oracle.copy_blocks(kp, vp, step.copy_pairs)
+    kp, vp = oracle.reshape_and_cache(raw_bits(step.new_key), raw_bits(step.new_value), kp, vp,
+                                      step.slot_mapping)
+    idx = torch.tensor(touched, dtype=torch.long, device="cuda")
+    got_k, got_v = raw_bits(kc.index_select(0, idx)), raw_bits(vc.index_select(0, idx))
+    for i, b in enumerate(touched):
+        assert np.array_equal(got_k[i], kp[b]) and np.array_equal(got_v[i], vp[b]), f"block {b}"
+    untouched = torch.ones(step.num_blocks, dtype=torch.bool, device="cuda")
+    untouched[idx] = False
+    assert torch.equal(kc[untouched], pre_k[untouched]) and torch.equal(vc[untouched], pre_v[untouched])
+    # decode: sampled sequences (shortest, longest and random ones), every head
+    rng = np.random.default_rng(0)
+    ctx = step.context_lens
+    seqs = sorted({int(np.argmin(ctx)), int(np.argmax(ctx))} |
+                  set(int(x) for x in rng.choice(step.num_seqs, size=min(4, step.num_seqs), replace=False)))
+    ref = oracle_outputs(step, seqs, pre_k, pre_v)
+    got = f64(out)
+    for s in seqs:
+        assert_close(got[s], ref[s], torch.bfloat16, torch.float32, f"{name} seq {s} ctx {ctx[s]}")
+
+
+# ---------------------------------------------------------------------------
+# invariants the pages fix, checked bit for bit on the GPU
+# ---------------------------------------------------------------------------
+
+def test_reservation_and_free_blocks_are_ignored(pa):
+    """NaN in every free block and reservation slot, -1 past each table's end:
+    the output equals the run without them, bit for bit, and is finite."""
+    kw = dict(dtype=torch.bfloat16, num_heads=16, num_kv_heads=4, head_dim=128, block_size=16, seed=21,
+              partition_size=64)
+    ctx = [1, 17, 100, 333, 64, 65]
+    clean = to_device(W.independent("clean", ctx, poison=False, **kw))
+    dirty = to_device(W.independent("dirty", ctx, poison=True, **kw))
+    a, *_ = run_gpu(pa, clean)
+    b, *_ = run_gpu(pa, dirty)
+    assert torch.isfinite(b).all()
+    assert torch.equal(a, b)
+
+
+def test_permutation_of_physical_blocks(pa):
+    step = to_device(W.independent("perm", [3, 95, 640, 17, 1100], dtype=torch.bfloat16, num_heads=32,
+                                   num_kv_heads=8, head_dim=128, block_size=16, seed=9, partition_size=128))
+    base, *_ = run_gpu(pa, step)
+    perm = np.random.default_rng(5).permutation(step.num_blocks)
+    inv = torch.from_numpy(np.argsort(perm)).cuda()
+    moved = W.DecodeStep(**{**step.__dict__})
+    moved.k_cache = step.k_cache[inv].contiguous()    # block b moves to perm[b]
+    moved.v_cache = step.v_cache[inv].contiguous()
+    moved.block_tables = np.where(step.block_tables >= 0, perm[np.maximum(step.block_tables, 0)], -1)
+    moved.slot_mapping = np.where(step.slot_mapping >= 0,
+                                  perm[step.slot_mapping // step.block_size] * step.block_size
+                                  + step.slot_mapping % step.block_size, -1)
+    again, *_ = run_gpu(pa, moved)
+    assert torch.equal(base, again)
+
+
+def test_deterministic_and_shared_tables(pa):
+    step = to_device(W.independent("det", [900, 900, 31], dtype=torch.bfloat16, num_heads=32,
+                                   num_kv_heads=8, head_dim=128, block_size=16, seed=4, partition_size=256))
+    step.q[1] = step.q[0]
+    tables = step.block_tables.copy()
+    tables[1] = tables[0]                  # sequence 1 reads sequence 0's blocks
+    slots = step.slot_mapping.copy()
+    slots[1] = -1                           # ... and writes nothing of its own
+    a, *_ = run_gpu(pa, step, tables=tables, slots=slots)
+    b, *_ = run_gpu(pa, step, tables=tables, slots=slots)
+    assert torch.equal(a, b)
+    assert torch.equal(a[0], a[1])
+
+
+def test_single_token_context_returns_the_value_row(pa):
+    step = to_device(W.independent("one", [1, 1, 1], dtype=torch.bfloat16, num_heads=8, num_kv_heads=2,
+                                   head_dim=128, block_size=8, seed=2))
+    out, kc, vc, _, _ = run_gpu(pa, step)
+    for s in range(3):
+        for h in range(8):
+            assert torch.equal(out[s, h], step.new_value[s, h // 4].float())
+
+
+# ---------------------------------------------------------------------------
+# data-dependent errors: skipped and reported, never a fault
+# ---------------------------------------------------------------------------
+
+def test_bad_block_id_is_flagged(pa):
+    step = to_device(W.independent("badblk", [40, 40], dtype=torch.bfloat16, num_heads=8, num_kv_heads=8,
+                                   head_dim=128, block_size=16, seed=6))
+    tables = step.block_tables.copy()
+    tables[0, 1] = step.num_blocks + 5
+    out, _, _, err, _ = run_gpu(pa, step, tables=tables)
+    assert err & pa.DEVERR_BLOCK_ID
+    assert torch.isfinite(out).all()
+    ref = full_oracle(step)
+    assert_close(f64(out[1]), ref[1], torch.bfloat16, torch.float32, "healthy sequence")
+
+
+def test_bad_block_id_fp32(pa):
+    step = to_device(W.tiny(block_size=4))
+    tables = step.block_tables.copy()
+    tables[3, 2] = -7
+    out, _, _, err, _ = run_gpu(pa, step, tables=tables)
+    assert err & pa.DEVERR_BLOCK_ID
+
+
+def test_bad_slot_and_pair_are_flagged(pa):
+    step = to_device(W.independent("badslot", [5, 9], dtype=torch.bfloat16, num_heads=4, num_kv_heads=4,
+                                   head_dim=64, block_size=4, seed=8))
+    slots = step.slot_mapping.copy()
+    slots[0] = step.num_blocks * step.block_size + 3
+    kc, vc = step.k_cache.clone(), step.v_cache.clone()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.reshape_and_cache(step.new_key, step.new_value, kc, vc, torch.from_numpy(slots).cuda(), dev_err=err)
+    pa.copy_blocks(kc, vc, torch.tensor([[0, step.num_blocks]], dtype=torch.int64, device="cuda"), dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() & pa.DEVERR_SLOT and err.item() & pa.DEVERR_COPY
+    # the valid token was still written, the invalid one and the bad copy were skipped
+    ek, _ = oracle.reshape_and_cache(raw_bits(step.new_key[1:]), raw_bits(step.new_value[1:]),
+                                     raw_bits(step.k_cache), raw_bits(step.v_cache), slots[1:])
+    assert np.array_equal(raw_bits(kc), ek)
+
+
+def test_context_above_capacity_is_clamped_and_flagged(pa):
+    step = to_device(W.independent("cap", [100, 20], dtype=torch.bfloat16, num_heads=8, num_kv_heads=8,
+                                   head_dim=128, block_size=16, seed=12))
+    out, _, _, err, _ = run_gpu(pa, step, max_context_len=64)
+    assert err & pa.DEVERR_CONTEXT
+    clamped = W.DecodeStep(**{**step.__dict__})
+    clamped.context_lens = np.minimum(step.context_lens, 64)
+    ref = full_oracle(clamped)
+    assert_close(f64(out), ref, torch.bfloat16, torch.float32, "clamped")

@@ -1,0 +1,120 @@
+"""CPU checks of the C ABI: libpa.so loads, exports every function include/pa.h
+declares, and rejects bad arguments on the host before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_382_b200 import build
+
+    build.build()
+    from paged_kv_cache_382_b200 import pa as binding
+
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(pa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["pa_reshape_and_cache", "pa_decode", "pa_decode_phases", "pa_decode_workspace_bytes",
+                     "pa_copy_blocks", "pa_status_string", "pa_version"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(pa):
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(declared_functions()) <= set(pa.SIGNATURES)
+
+
+def test_status_strings_and_version(pa):
+    assert pa.lib.pa_status_string(0).decode() == "PA_OK"
+    assert b"workspace" in pa.lib.pa_status_string(3)
+    assert pa.lib.pa_version() >= 100
+
+
+def test_workspace_bytes(pa):
+    ws = pa.lib.pa_decode_workspace_bytes
+    # one partition: header + work list only
+    assert ws(64, 32, 128, 512, 512) == 256 + 256
+    # several partitions: + (max, sum) and the fp32 partial outputs
+    S, H, D, cap, P = 8, 64, 128, 131072, 512
+    parts = cap // P
+    expect = 256 + (S * parts * 4 + 255) // 256 * 256 + (S * H * parts * 8 + 255) // 256 * 256 \
+        + (S * H * parts * D * 4 + 255) // 256 * 256
+    assert ws(S, H, D, cap, P) == expect
+    assert ws(-1, 1, 64, 10, 512) == 0
+    assert ws(1, 1, 64, 10, 0) == 0
+
+
+def _decode_call(pa, **over):
+    args = dict(out=1 << 20, out_dtype=0, q=1 << 20, k=1 << 20, v=1 << 20, tables=1 << 20, ctx=1 << 20,
+                S=4, Hq=4, Hkv=4, D=64, B=16, NB=64, max_blocks=8, max_ctx=0, scale=0.125, P=512,
+                ws=1 << 20, ws_bytes=1 << 30, dtype=0, err=None, stream=None, phases=7)
+    args.update(over)
+    return pa.lib.pa_decode_phases(args["out"], args["out_dtype"], args["q"], args["k"], args["v"],
+                                   args["tables"], args["ctx"], args["S"], args["Hq"], args["Hkv"],
+                                   args["D"], args["B"], args["NB"], args["max_blocks"], args["max_ctx"],
+                                   args["scale"], args["P"], args["ws"], args["ws_bytes"], args["dtype"],
+                                   args["err"], args["stream"], args["phases"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(Hq=6, Hkv=4), 1),            # heads not a multiple of kv heads
+    (dict(D=96), 2),                   # head_dim
+    (dict(B=64), 2),                   # block_size
+    (dict(P=48), 2),                   # partition not a multiple of 32
+    (dict(P=16384), 2),                # partition too large
+    (dict(B=32, P=32 + 32 * 0), 0),    # fine shapes, but S=0 below
+    (dict(dtype=5), 1),                # dtype
+    (dict(out_dtype=1, dtype=0), 2),   # bf16 output from fp32 input
+    (dict(ws=None), 1),                # no workspace
+    (dict(ws=(1 << 20) + 8), 1),       # misaligned workspace
+    (dict(ws_bytes=10), 3),            # short workspace
+    (dict(q=(1 << 20) + 2), 1),        # misaligned q
+    (dict(tables=None), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(phases=0), 1),
+    (dict(phases=8), 1),
+    (dict(max_ctx=-1), 1),
+])
+def test_decode_host_validation(pa, over, status):
+    if status == 0:
+        over = dict(over, S=0)          # an empty batch is a no-op that touches nothing
+    assert _decode_call(pa, **over) == status
+
+
+def test_cache_ops_host_validation(pa):
+    L = pa.lib
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, 8, 128, 16, 64, 1, None, None) == 0
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 3, 8, 128, 16, 64, 1, None, None) == 1
+    assert L.pa_reshape_and_cache(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 3, 8, 80, 16, 64, 1, None,
+                                  None) == 2
+    assert L.pa_reshape_and_cache(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 3, 8, 128, 12, 64, 1, None,
+                                  None) == 2
+    assert L.pa_copy_blocks(None, None, None, 0, 4096, 64, None, None) == 0
+    assert L.pa_copy_blocks(None, None, None, 2, 4096, 64, None, None) == 1
+    assert L.pa_copy_blocks(1 << 20, 1 << 20, 1 << 20, 2, 4095, 64, None, None) == 1
+
+
+def test_binding_marshals_no_cpu_tensors(pa):
+    import torch
+
+    k = torch.zeros(4, 2, 16, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.reshape_and_cache(torch.zeros(1, 2, 64), torch.zeros(1, 2, 64), k, k.clone(),
+                             torch.zeros(1, dtype=torch.int64))
