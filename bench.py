@@ -1,0 +1,630 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged decode-attention hot path on B200 (sm_100a).
+
+One step = one decode step of one layer over a synthetic batch already resident
+in HBM, all through libpa's C ABI:
+  1. copy-on-write block copies (when the workload plans any),
+  2. scatter of the step's new K/V into the paged pool (one token per sequence),
+  3. paged decode attention: plan, attend, partition merge.
+
+Metric: paged decode attention KV GB/s (algorithmic bytes / step time; also as
+% of 8 TB/s and of the measured HBM copy bandwidth) and seq-tokens/s per layer
+(context tokens attended per second).  Algorithmic bytes of a step:
+  sum_s ctx_s*Hkv*d*2*e + 2*S*Hq*d*e + sum_s ceil(ctx_s/B)*4 + 4*S
+(shared prefix blocks counted once).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Default workload: Llama-7B-like decode layer in bf16 (64 sequences, 32 = 32
+heads, head_dim 128, block_size 16, context lengths uniform [128, 2048], an
+8192-block pool popped from a shuffled free list) plus the scatter of 64 new
+tokens.  Its K/V (1.16 GB per step) is far larger than the 126 MB L2, so no L2
+flush is needed between steps.  With N > 1 ranks (torchrun) every rank runs its
+own batch (seed + rank): weak scaling, no collective on the data path.
+
+Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s (% of 8 TB/s HBM) and seq-tokens/s per layer"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+CONFIGS = {
+    "llama7b": dict(builder="llama7b", kwargs={},
+                    desc="Llama-7B-like decode layer bf16: 64 seqs, 32 q = 32 kv heads, head_dim 128, "
+                         "block_size 16, context lens uniform [128, 2048], 8192-block shuffled pool, "
+                         "+ reshape_and_cache of 64 new tokens"),
+    "gqa": dict(builder="gqa", kwargs={},
+                desc="GQA decode bf16: 256 seqs, 32 q / 8 kv heads, head_dim 128, block_size 16, "
+                     "context lens log-normal (median 1000, sigma 1.0, capped 8192), 90% occupied pool"),
+    "shared_prefix": dict(builder="shared_prefix", kwargs=dict(prompt_len=512, suffix_max=512),
+                          desc="parallel sampling bf16: 16 prompts x 8 samples, 512-token prompt in "
+                               "shared blocks, suffix uniform [0, 512], 32 q / 8 kv heads, head_dim 128"),
+    "shared_prefix_cow": dict(builder="shared_prefix", kwargs=dict(prompt_len=520, suffix_max=0),
+                              desc="parallel sampling bf16, first decode step after a 520-token prompt: "
+                                   "112 copy-on-write block copies, 32 q / 8 kv heads, head_dim 128"),
+    "long_context_b8": dict(builder="long_context", kwargs=dict(block_size=8),
+                            desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
+                                 "64 q / 8 kv heads, head_dim 128, block_size 8, partitions of 512"),
+    "long_context_b16": dict(builder="long_context", kwargs=dict(block_size=16),
+                             desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
+                                  "64 q / 8 kv heads, head_dim 128, block_size 16, partitions of 512"),
+    "long_context_b32": dict(builder="long_context", kwargs=dict(block_size=32),
+                             desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
+                                  "64 q / 8 kv heads, head_dim 128, block_size 32, partitions of 512"),
+}
+DEFAULT_CONFIG = "llama7b"
+ATTEND_SOURCES = ["paged_kv_cache_382_b200/csrc/decode.cu", "paged_kv_cache_382_b200/csrc/pa_device.cuh"]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", choices=sorted(CONFIGS), default=DEFAULT_CONFIG)
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--partition-size", type=int, default=512)
+    p.add_argument("--cpu-core-seconds", type=float, default=15.0,
+                   help="CPU work of the oracle baseline sample, in core-seconds")
+    p.add_argument("--reference-seconds", type=float, default=150.0,
+                   help="wall-time budget of the whole --impl reference run")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# small helpers (no torch at module level: spawned oracle workers import this file)
+# ---------------------------------------------------------------------------
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def attend_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in ATTEND_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(config: str):
+    """dram bytes per attend launch from the committed ncu summary of this workload,
+    or None if there is none or the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"attend_{config}.ncu.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.lstrip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    try:
+        if fields.get("kernel_source_sha256") != attend_source_hash():
+            return None
+        return int(float(fields["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_id: str, enabled: bool = True):
+        self.device_id = device_id
+        self.enabled = enabled
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        if self.enabled:
+            fd, self.path = tempfile.mkstemp(prefix="pa_clocks_", suffix=".csv")
+            os.close(fd)
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.device_id}", f"--query-gpu={self.QUERY}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                time.sleep(0.3)
+            except OSError:
+                self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], None, set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, flag in zip(self.REASONS, parts[5:9]):
+                    if flag.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm): spawn workers, fp64 numpy
+# ---------------------------------------------------------------------------
+
+def _oracle_task(task):
+    """Runs in a spawned worker: decode attention of one sequence by the oracle,
+    over its blocks stored as .npy files (table = their order)."""
+    import numpy as np
+
+    import oracle
+
+    kpath, vpath, q, ctx, scale = task
+    k = np.load(kpath, mmap_mode="r")
+    v = np.load(vpath, mmap_mode="r")
+    table = np.arange(k.shape[0])[None]
+    t0 = time.perf_counter()
+    oracle.decode_attention(q[None], k, v, table, np.array([ctx]), scale)
+    return time.perf_counter() - t0
+
+
+class OracleSample:
+    """Stages the blocks of some sequences of a step on the host (not timed) and
+    times the oracle over them with a process pool of the machine's host cores."""
+
+    def __init__(self, step, seqs, pool, tmpdir):
+        import numpy as np
+        import torch
+
+        self.step, self.seqs, self.pool = step, list(seqs), pool
+        self.tasks = []
+        B = step.block_size
+        for s in self.seqs:
+            c = int(step.context_lens[s])
+            ids = torch.from_numpy(step.block_tables[s, : -(-c // B)].astype(np.int64)).to(step.k_cache.device)
+            kp = os.path.join(tmpdir, f"k{s}.npy")
+            vp = os.path.join(tmpdir, f"v{s}.npy")
+            np.save(kp, step.k_cache.index_select(0, ids).float().cpu().numpy())
+            np.save(vp, step.v_cache.index_select(0, ids).float().cpu().numpy())
+            q = step.q[s].double().cpu().numpy()
+            self.tasks.append((kp, vp, q, c, step.scale))
+
+    def bytes(self):
+        st = self.step
+        e = st.element_bytes
+        kv = sum(int(st.context_lens[s]) for s in self.seqs) * st.num_kv_heads * st.head_dim * 2 * e
+        qo = 2 * len(self.seqs) * st.num_heads * st.head_dim * e
+        tb = sum(-(-int(st.context_lens[s]) // st.block_size) for s in self.seqs) * 4 + 4 * len(self.seqs)
+        return kv + qo + tb
+
+    def tokens(self):
+        return sum(int(self.step.context_lens[s]) for s in self.seqs)
+
+    def run(self, repeats=1):
+        t0 = time.perf_counter()
+        busy = 0.0
+        for _ in range(repeats):
+            busy += sum(self.pool.map(_oracle_task, self.tasks, chunksize=1))
+        return time.perf_counter() - t0, busy
+
+
+def make_oracle_pool():
+    import multiprocessing as mp
+
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    os.environ.setdefault("OPENBLAS_NUM_THREADS", "1")
+    os.environ.setdefault("MKL_NUM_THREADS", "1")
+    cores = len(os.sched_getaffinity(0))
+    return mp.get_context("spawn").Pool(cores), cores
+
+
+# ---------------------------------------------------------------------------
+# the GPU path
+# ---------------------------------------------------------------------------
+
+class DeviceStep:
+    """One step's inputs resident on the device plus the preallocated outputs."""
+
+    def __init__(self, pa, step, partition_size):
+        import numpy as np
+        import torch
+
+        dev = step.k_cache.device
+        self.pa, self.step = pa, step
+        self.kc, self.vc = step.k_cache, step.v_cache
+        self.q, self.new_key, self.new_value = step.q, step.new_key, step.new_value
+        self.slots = torch.from_numpy(step.slot_mapping).to(dev)
+        self.pairs = torch.from_numpy(np.ascontiguousarray(step.copy_pairs)).to(dev)
+        self.tables = torch.from_numpy(step.block_tables.astype(np.int32)).to(dev)
+        self.ctx = torch.from_numpy(step.context_lens.astype(np.int32)).to(dev)
+        self.out = torch.empty(step.num_seqs, step.num_heads, step.head_dim, dtype=step.dtype, device=dev)
+        self.P = partition_size
+        self.cap = pa.decode_capacity(self.tables, step.block_size, step.max_context_len)
+        self.ws = pa.alloc_workspace(step.num_seqs, step.num_heads, step.head_dim, self.cap, partition_size,
+                                     dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.launches_per_step = (1 if len(step.copy_pairs) else 0) + 1 + 3
+
+    def run(self, ev_attend=None, q=None, new_key=None, new_value=None, slots=None, tables=None, ctx=None,
+            out=None):
+        pa = self.pa
+        if len(self.step.copy_pairs):
+            pa.copy_blocks(self.kc, self.vc, self.pairs, dev_err=self.err)
+        pa.reshape_and_cache(new_key if new_key is not None else self.new_key,
+                             new_value if new_value is not None else self.new_value,
+                             self.kc, self.vc, slots if slots is not None else self.slots, dev_err=self.err)
+        args = (out if out is not None else self.out, q if q is not None else self.q, self.kc, self.vc,
+                tables if tables is not None else self.tables, ctx if ctx is not None else self.ctx,
+                self.step.scale)
+        kw = dict(max_context_len=self.cap, partition_size=self.P, workspace=self.ws, dev_err=self.err)
+        pa.decode(*args, phases=pa.PHASE_PLAN, **kw)
+        if ev_attend is not None:
+            ev_attend[0].record()
+        pa.decode(*args, phases=pa.PHASE_ATTEND, **kw)
+        if ev_attend is not None:
+            ev_attend[1].record()
+        pa.decode(*args, phases=pa.PHASE_REDUCE, **kw)
+
+
+def nvsmi_id(local_index: int) -> str:
+    """nvidia-smi's name for torch device ``local_index`` (its UUID), robust to
+    CUDA_VISIBLE_DEVICES remapping."""
+    import torch
+
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(local_index).uuid)
+    except Exception:
+        return str(local_index)
+
+
+def build_step(config: str, seed: int, device, partition_size: int):
+    from paged_kv_cache_382_b200 import workloads as W
+
+    spec = CONFIGS[config]
+    fn = W.WORKLOADS[spec["builder"]]
+    return fn(seed=seed, device=device, partition_size=partition_size, **spec["kwargs"])
+
+
+def dist_setup():
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def reduce_over_ranks(values, ops):
+    """All-reduce a few scalars over the ranks (SUM or MAX each); identity at N=1."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return list(values)
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else "cpu"
+    out = []
+    for v, op in zip(values, ops):
+        t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+        out.append(float(t.item()))
+    return out
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_382_b200 import build as _build
+    from paged_kv_cache_382_b200 import workloads as W
+
+    world, rank, local = dist_setup()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    # the oracle pool is spawned before any CUDA work
+    pool = cores = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        pool, cores = make_oracle_pool()
+    _build.build()
+    from paged_kv_cache_382_b200 import pa
+
+    dev = torch.device("cuda", local)
+    step = build_step(args.config, args.seed + rank, dev, args.partition_size)
+    ds = DeviceStep(pa, step, args.partition_size)
+    alg_bytes = W.algorithmic_bytes(step, unique=True)
+    logical_bytes = W.algorithmic_bytes(step, unique=False)
+    ctx_tokens = int(step.context_lens.sum())
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        ds.run()
+    torch.cuda.synchronize()
+    if int(ds.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(ds.err.item()):#x}")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(nvsmi_id(local), enabled=not args.no_clocks) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            ds.run(ev_attend=ev[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    attend_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    clock_info = clocks.summary()
+
+    # end to end through the public API: host inputs in, host result out, every step
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(ds, step, alg_bytes, max(args.warmup, 3), min(K, 1000))
+
+    tot_bytes, max_ms, tot_tokens, tot_seqs = reduce_over_ranks(
+        [alg_bytes * K, elapsed_ms, ctx_tokens * K, step.num_seqs * K], ["sum", "max", "sum", "sum"])
+    if e2e is not None:
+        e2e_bytes, e2e_ms = reduce_over_ranks([e2e["bytes"], e2e["ms"]], ["sum", "max"])
+    peak, peak_kind = measured_hbm_peak()
+    achieved_attend = alg_bytes / (attend_ms * 1e-3) / 1e9
+    value = tot_bytes / (max_ms * 1e-3) / 1e9
+
+    cpu = None
+    if pool is not None:
+        cpu = cpu_baseline(step, pool, cores, args.cpu_core_seconds)
+        pool.close()
+    if rank != 0:
+        return
+    traffic = profiled_traffic(args.config)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": round(max_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if step.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded; K/V ~ N(0,1) generated on the device by torch, no dataset)",
+        "config": {
+            "workload": CONFIGS[args.config]["desc"],
+            "name": args.config,
+            "num_seqs_per_gpu": step.num_seqs,
+            "context_tokens_per_gpu": ctx_tokens,
+            "partition_size": args.partition_size,
+            "parallelism": f"replicas x{world} (independent batches, no collective)",
+            "l2": f"inputs larger than L2: {alg_bytes / 1e9:.3f} GB of K/V+q/out per step vs 126 MB L2",
+        },
+        "pct_of_8tbs": round(100.0 * value / NOMINAL_HBM_GBS, 2),
+        "pct_of_measured_hbm": round(100.0 * value / peak, 2),
+        "seq_tokens_per_s": round(tot_tokens / (max_ms * 1e-3), 1),
+        "decode_tokens_per_s": round(tot_seqs / (max_ms * 1e-3), 1),
+        "algorithmic_bytes_per_step": alg_bytes,
+        "logical_bytes_per_step": logical_bytes,
+        "effective_logical_gbs": round(logical_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
+        "gpu_launches": ds.launches_per_step * K,
+        "roofline": {
+            "kernel": "attend_bf16_kernel" if step.dtype == torch.bfloat16 else "attend_f32_kernel",
+            "bound": "hbm",
+            "achieved": round(achieved_attend, 2),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+            "unit": "GB/s",
+            "frac": round(achieved_attend / peak, 4),
+            "traffic": traffic,
+            "attend_ms": round(attend_ms, 5),
+            "bytes_per_launch": alg_bytes,
+        },
+        "clocks": clock_info,
+        "e2e": None,
+        "cpu_baseline": cpu,
+    }
+    if e2e is not None:
+        line["e2e"] = {"value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e_ms / e2e["steps"], 5), "steps": e2e["steps"]}
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(ds, step, alg_bytes, warmup, steps):
+    """Same step through the binding with the step's inputs in pinned host memory:
+    H2D of q / new K,V / slots / tables / context lens, the step, D2H of out."""
+    import torch
+
+    host = {name: t.cpu().pin_memory() for name, t in dict(
+        q=ds.q, new_key=ds.new_key, new_value=ds.new_value, slots=ds.slots, tables=ds.tables,
+        ctx=ds.ctx).items()}
+    dev = {name: torch.empty_like(t, device=ds.q.device) for name, t in host.items()}
+    out_host = torch.empty(ds.out.shape, dtype=ds.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one():
+        for name in host:
+            dev[name].copy_(host[name], non_blocking=True)
+        ds.run(q=dev["q"], new_key=dev["new_key"], new_value=dev["new_value"], slots=dev["slots"],
+               tables=dev["tables"], ctx=dev["ctx"])
+        out_host.copy_(ds.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        one()
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    return {"ms": start.elapsed_time(stop), "bytes": alg_bytes * steps, "h2d": h2d, "d2h": d2h,
+            "steps": steps}
+
+
+def cpu_baseline(step, pool, cores, core_seconds):
+    """The oracle timed on the host cores over a bounded sample of the same batch."""
+    with tempfile.TemporaryDirectory(prefix="pa_oracle_") as tmp:
+        sample = OracleSample(step, range(step.num_seqs), pool, tmp)
+        wall1, busy1 = sample.run(1)            # first pass also warms the workers
+        repeats = max(1, int(math.ceil(core_seconds / max(busy1, 1e-3))))
+        wall, busy = sample.run(repeats)
+        return {
+            "value": round(sample.bytes() * repeats / wall / 1e9, 4),
+            "unit": UNIT,
+            "cores": cores,
+            "kind": "oracle",
+            "sample": f"all {len(sample.seqs)} sequences of the batch (every head, "
+                      f"{sample.tokens()} context tokens) x {repeats} passes, decode attention only, "
+                      f"fp64 numpy, one sequence per task; {busy:.1f} core-s of work in {wall:.2f} s",
+            "seq_tokens_per_s": round(sample.tokens() * repeats / wall, 1),
+        }
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    pool, cores = make_oracle_pool()
+    import torch
+
+    from paged_kv_cache_382_b200 import workloads as W
+
+    del W
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))) if torch.cuda.is_available() else "cpu"
+    step = build_step(args.config, args.seed, dev, args.partition_size)
+    with tempfile.TemporaryDirectory(prefix="pa_oracle_") as tmp:
+        full = OracleSample(step, range(step.num_seqs), pool, tmp)
+        wall1, busy1 = full.run(1)
+        per_seq = busy1 / len(full.seqs)
+        # sequences per step so that warmup + steps fit the time budget
+        n_steps = max(args.warmup, 3) + args.steps
+        per_step_budget = args.reference_seconds / n_steps
+        n_seq = max(1, min(len(full.seqs), int(per_step_budget * cores / max(per_seq, 1e-6))))
+        total_wall, total_bytes, total_tokens = 0.0, 0, 0
+        for i in range(n_steps):
+            seqs = [(i * n_seq + j) % len(full.seqs) for j in range(n_seq)]
+            sub = OracleSample.__new__(OracleSample)
+            sub.step, sub.seqs, sub.pool = step, seqs, pool
+            sub.tasks = [full.tasks[s] for s in seqs]
+            wall, _ = sub.run(1)
+            if i >= max(args.warmup, 3):
+                total_wall += wall
+                total_bytes += sub.bytes()
+                total_tokens += sub.tokens()
+    pool.close()
+    value = total_bytes / total_wall / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": round(1e3 * total_wall / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded, same batch as the GPU arm)",
+        "config": {"workload": CONFIGS[args.config]["desc"], "name": args.config},
+        "seq_tokens_per_s": round(total_tokens / total_wall, 1),
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{n_seq} of {len(full.seqs)} sequences per step (every head), "
+                                   f"decode attention by the fp64 numpy oracle, one sequence per task"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    try:
+        import torch.distributed as dist
+
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+if __name__ == "__main__":
+    main()
