@@ -182,6 +182,41 @@ int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k
 int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
                    size_t block_bytes, int num_blocks, int32_t* dev_err, pa_stream stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for such callers:
+ * a host program whose device memory is planned once at start-up (the KV pool
+ * takes nearly all of HBM and nothing may be allocated while serving), a
+ * latency-critical caller that must not pay cudaMalloc/cudaFree and the device
+ * synchronisation they imply, or a foreign-language caller that links only this
+ * C ABI and has no CUDA allocator at hand.
+ *
+ * Arguments and results are those of pa_decode minus the workspace: instead of a
+ * caller workspace it uses a fixed array of PA_NOALLOC_SCRATCH_BYTES inside the
+ * library.  It allocates nothing and calls no allocating routine; inputs and
+ * outputs remain the caller's.
+ *  - Limit: a batch that needs more than PA_NOALLOC_SCRATCH_BYTES (what
+ *    pa_decode_workspace_bytes() returns for the same context bound pa_decode
+ *    uses) is rejected with PA_ERR_WORKSPACE and nothing is launched.
+ *  - Memory: every GPU on which the library loads the array holds those bytes
+ *    until the process exits.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    with that device current and caches it; make that first call before any
+ *    stream capture.
+ *  - Sharing: all calls on a device use the same array, which keeps the last
+ *    call's contents.  Nothing in it has to start at zero -- each call rewrites
+ *    its work list and count and reads only partials it wrote itself -- but calls
+ *    whose kernels overlap on the GPU (other streams, other host threads) race on
+ *    it: serialise them.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int num_seqs, int num_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      int max_blocks_per_seq, int max_context_len, float scale,
+                      int partition_size, pa_dtype dtype, int32_t* dev_err, pa_stream stream);
+
 /* Human-readable name of a pa_status value (static storage). */
 const char* pa_status_string(int status);
 

@@ -35,6 +35,8 @@ SIGNATURES = {
     "pa_decode": (_i, _DECODE_ARGS),
     "pa_decode_phases": (_i, _DECODE_ARGS + [_i]),
     "pa_copy_blocks": (_i, [_vp, _vp, _i64p, _i, _sz, _i, _i32p, _vp]),
+    "pa_decode_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i32p, _i32p, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                               _i, _i, _i32p, _vp]),
     "pa_status_string": (ctypes.c_char_p, [_i]),
     "pa_version": (_i, []),
 }
@@ -182,3 +184,27 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: tor
                             _dev(src_dst_pairs, "src_dst_pairs", torch.int64), n, block_bytes,
                             k_cache.shape[0], _opt_err(dev_err), _stream_handle(stream))
     _check(rc, "pa_copy_blocks")
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, *,
+                   max_context_len: int = 0, partition_size: int = 512,
+                   dev_err: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Paged decode attention for callers that cannot allocate device memory: like
+    ``decode`` but with the workspace in a fixed 64 MiB array inside the library
+    (shared by all calls on a device; calls that overlap on the GPU race)."""
+    NB, Hkv, B, d = k_cache.shape
+    S, Hq, _ = q.shape
+    dt = k_cache.dtype
+    rc = lib.pa_decode_noalloc(
+        _dev(out, "out"), dtype_code(out.dtype), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt),
+        _dev(v_cache, "v_cache", dt), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), S, Hq, Hkv, d, B, NB, block_tables.shape[1],
+        max_context_len, float(scale), partition_size, dtype_code(dt), _opt_err(dev_err),
+        _stream_handle(stream))
+    _check(rc, "pa_decode_noalloc")
+    return out
