@@ -49,6 +49,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* Only the entry points below are exported from libpa.so. */
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -92,7 +99,7 @@ typedef void* pa_stream;        /* a cudaStream_t */
  * The copy is bit-exact.  Two tokens naming the same slot race (caller error).
  * num_tokens == 0 is a no-op.
  */
-int pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+PA_API int pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
                          const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                          int head_dim, int block_size, int num_blocks, pa_dtype dtype,
                          int32_t* dev_err, pa_stream stream);
@@ -106,7 +113,7 @@ int pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void
  * one (max, sum, unnormalised output) partial per sequence, head and partition
  * in fp32.  Its contents need no initialisation.
  */
-size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+PA_API size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                  int max_context_len, int partition_size);
 
 /*
@@ -136,7 +143,7 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
  * bit-identical under any renumbering of physical blocks and run to run.
  * Launches three kernels (plan, attention, merge) on `stream`.
  */
-int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+PA_API int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
               const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
               int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
               int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
@@ -157,7 +164,7 @@ int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
 #define PA_PHASE_ATTEND 0x2
 #define PA_PHASE_REDUCE 0x4
 #define PA_PHASE_ALL    0x7
-int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+PA_API int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
                      const void* v_cache, const int32_t* block_tables,
                      const int32_t* context_lens, int num_seqs, int num_heads,
                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
@@ -179,7 +186,7 @@ int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k
  *                 size; a positive multiple of 16.
  * The copy is bit-exact.  num_pairs == 0 is a no-op.
  */
-int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
+PA_API int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
                    size_t block_bytes, int num_blocks, int32_t* dev_err, pa_stream stream);
 
 /*
@@ -210,7 +217,7 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, i
  *    it: serialise them.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
-int pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+PA_API int pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* block_tables,
                       const int32_t* context_lens, int num_seqs, int num_heads,
                       int num_kv_heads, int head_dim, int block_size, int num_blocks,
@@ -218,10 +225,10 @@ int pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* q, const void* 
                       int partition_size, pa_dtype dtype, int32_t* dev_err, pa_stream stream);
 
 /* Human-readable name of a pa_status value (static storage). */
-const char* pa_status_string(int status);
+PA_API const char* pa_status_string(int status);
 
 /* Library version: major*10000 + minor*100 + patch. */
-int pa_version(void);
+PA_API int pa_version(void);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB_PATH = os.path.join(HERE, "libpa.so")
 SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
-DEPS = SOURCES + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")) +
+DEPS = SOURCES + [os.path.abspath(__file__)] + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")) +
                         glob.glob(os.path.join(HERE, "csrc", "*.h")) +
                         glob.glob(os.path.join(ROOT, "include", "*.h")))
 
@@ -46,7 +46,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB_PATH
     tmp = LIB_PATH + ".tmp"
     cmd = [nvcc_path(), "-O3", "-std=c++17", *ARCH_FLAGS, "-lineinfo",
-           "-Xcompiler", "-fPIC,-O2", "-shared", "-I", os.path.join(ROOT, "include"),
+           "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden", "-shared", "-I", os.path.join(ROOT, "include"),
            "-o", tmp, *SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")

@@ -21,6 +21,8 @@ reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict_
                          uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                          const int64_t* __restrict__ slot_mapping, int num_kv_heads, int row_vecs,
                          int block_size, int64_t num_slots, int32_t* dev_err) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int t = blockIdx.x;
     const int64_t slot = slot_mapping[t];
     if (slot < 0) return;
@@ -47,6 +49,8 @@ __global__ void __launch_bounds__(256)
 copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                    const int64_t* __restrict__ pairs, int64_t block_vecs, int num_blocks,
                    int32_t* dev_err) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int64_t src = pairs[2 * static_cast<int64_t>(blockIdx.y)];
     const int64_t dst = pairs[2 * static_cast<int64_t>(blockIdx.y) + 1];
     if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -88,11 +92,11 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
     const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
     const int per_token = num_kv_heads * row_vecs;
     const int threads = per_token >= 256 ? 256 : ((per_token + 31) / 32) * 32;
-    reshape_and_cache_kernel<<<num_tokens, threads, 0, as_stream(stream)>>>(
-        static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(k_cache),
-        static_cast<uint4*>(v_cache), slot_mapping, num_kv_heads, row_vecs, block_size, num_slots,
-        dev_err);
-    return launch_status();
+    return launch_status(launch_pdl(reshape_and_cache_kernel, dim3(num_tokens), dim3(threads), 0,
+                                    as_stream(stream), static_cast<const uint4*>(key),
+                                    static_cast<const uint4*>(value), static_cast<uint4*>(k_cache),
+                                    static_cast<uint4*>(v_cache), slot_mapping, num_kv_heads, row_vecs,
+                                    block_size, num_slots, dev_err));
 }
 
 extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,
@@ -112,10 +116,9 @@ extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_d
     if (ctas < 1) ctas = 1;
     if (ctas > 1024) ctas = 1024;
     dim3 grid(static_cast<unsigned>(ctas), static_cast<unsigned>(num_pairs));
-    copy_blocks_kernel<<<grid, threads, 0, as_stream(stream)>>>(
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), src_dst_pairs, block_vecs,
-        num_blocks, dev_err);
-    return launch_status();
+    return launch_status(launch_pdl(copy_blocks_kernel, grid, dim3(threads), 0, as_stream(stream),
+                                    static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                                    src_dst_pairs, block_vecs, num_blocks, dev_err));
 }
 
 extern "C" const char* pa_status_string(int status) {

@@ -24,7 +24,12 @@
 //               A sequence that fits one partition writes its output directly;
 //               otherwise each partition writes (max, sum, unnormalised
 //               output) to the workspace.
-//   3. reduce:  merges the partitions of each (seq, head) in partition order.
+//   3. reduce:  merges the partitions of each multi-partition (seq, head), in a
+//               fixed order (launched only when a context can span several
+//               partitions).
+// Every kernel is launched with programmatic dependent launch: it may start
+// while its predecessor in the stream finishes, and waits for it
+// (griddepcontrol.wait) before touching global memory.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -108,17 +113,36 @@ __device__ int cta_exclusive_scan(int v, int* total, int* scratch) {
 
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
     __shared__ int scratch[33];
+    pdl_wait();
+    pdl_launch_dependents();
     const int P = a.partition_size;
-    int nf = 0, nt = 0;
-    bool bad = false;
-    for (int s = threadIdx.x; s < a.num_seqs; s += PLAN_THREADS) {
+    // an item per whole partition, then one per ragged tail; an empty context
+    // is one item that writes zeros
+    auto counts = [&](int s, int& f, int& t) {
         const int raw = a.context_lens[s];
         const int c = clamp_context(raw, a.cap);
-        bad |= (c != raw);
-        nf += c / P;
-        nt += (c % P) != 0;
+        if (c != raw) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
+        f = c / P;
+        t = (c % P) != 0 || c == 0;
+    };
+    if (a.num_seqs <= PLAN_THREADS) {   // one pass
+        const int s = threadIdx.x;
+        int f = 0, t = 0, full_total = 0, tail_total = 0;
+        if (s < a.num_seqs) counts(s, f, t);
+        const int ef = cta_exclusive_scan(f, &full_total, scratch);
+        const int et = cta_exclusive_scan(t, &tail_total, scratch);
+        for (int k = 0; k < f; ++k) a.ws_items[ef + k] = s * a.max_parts + k;
+        if (t) a.ws_items[full_total + et] = s * a.max_parts + f;
+        if (threadIdx.x == 0) *a.ws_count = full_total + tail_total;
+        return;
     }
-    if (bad) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
+    int nf = 0, nt = 0;
+    for (int s = threadIdx.x; s < a.num_seqs; s += PLAN_THREADS) {
+        int f, t;
+        counts(s, f, t);
+        nf += f;
+        nt += t;
+    }
     int full_total = 0, tail_total = 0;
     cta_exclusive_scan(nf, &full_total, scratch);
     cta_exclusive_scan(nt, &tail_total, scratch);
@@ -129,7 +153,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
         if (s < a.num_seqs) {
             const int c = clamp_context(a.context_lens[s], a.cap);
             f = c / P;
-            t = (c % P) != 0;
+            t = (c % P) != 0 || c == 0;
         }
         int chunk_f = 0, chunk_t = 0;
         const int ef = cta_exclusive_scan(f, &chunk_f, scratch);
@@ -167,7 +191,7 @@ __device__ __forceinline__ void combine_store(const DecodeArgs& a, const float* 
             }
         }
         const size_t row = static_cast<size_t>(s) * a.num_heads + head0 + n;
-        if (nparts == 1) {
+        if (nparts <= 1) {
             const float v = L > 0.f ? O / L : 0.f;
             if (a.out_f32)
                 static_cast<float*>(a.out)[row * D + d] = v;
@@ -202,8 +226,14 @@ struct TileGeom {
     }
 };
 
+// Resident CTAs per SM the bf16 attend kernel is register-budgeted for (shared
+// memory allows 4 at 3 warps x 2 stages).
+#ifndef PA_ATTEND_MIN_CTAS
+#define PA_ATTEND_MIN_CTAS 4
+#endif
+
 template <int D, int RB, int W, int NS>
-__global__ void __launch_bounds__(W * 32)
+__global__ void __launch_bounds__(W * 32, PA_ATTEND_MIN_CTAS)
 attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const DecodeArgs a) {
     using Geo = TileGeom<D, RB>;
@@ -230,6 +260,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
     fence_barrier_init();
     __syncthreads();
+    pdl_wait();               // the work list is written by the plan kernel
+    pdl_launch_dependents();
 
     const int per_item = a.num_kv_heads * a.head_groups;
     const long long units = static_cast<long long>(*a.ws_count) * per_item;
@@ -264,7 +296,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int t1 = min(t0 + P, ctx);
         const int ntok = t1 - t0;
         const int nparts = (ctx + P - 1) / P;
-        const int nblk = (t1 - 1) / B - t0 / B + 1;
+        const int nblk = ntok > 0 ? (t1 - 1) / B - t0 / B + 1 : 0;
         const int gsub = min(8, a.group - hg * 8);
         const int head0 = kvh * a.group + hg * 8;
 
@@ -373,14 +405,19 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 __syncwarp();
             }
 
-            // S^T (16 tokens x 8 heads) = K (16 x D) . Q^T (D x 8)
-            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+            // S^T (16 tokens x 8 heads) = K (16 x D) . Q^T (D x 8), as two independent
+            // accumulation chains (even / odd k-steps) to halve the MMA dependency chain
+            float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                uint32_t a0, a1, a2, a3;
+            for (int ks = 0; ks < KS; ks += 2) {
+                uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
                 ldmatrix_x4(st + (ks / 4) * HALF + krow + kx[ks % 4], a0, a1, a2, a3);
+                ldmatrix_x4(st + ((ks + 1) / 4) * HALF + krow + kx[(ks + 1) % 4], e0, e1, e2, e3);
                 mma_bf16_16816(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                mma_bf16_16816(sd, e0, e1, e2, e3, qf[ks + 1][0], qf[ks + 1][1]);
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sc[i] += sd[i];
             // logits in the log2 domain; rows g and g+8 are tokens, columns 2c, 2c+1 heads
             float x0 = sc[0] * sl2, x1 = sc[1] * sl2, x2 = sc[2] * sl2, x3 = sc[3] * sl2;
             if (mask != 0xffffu) {
@@ -478,11 +515,13 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // ---------------------------------------------------------------------------
 
 template <int D>
-__global__ void __launch_bounds__(128) attend_f32_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) {
     constexpr int W = 4, J = D / 32;
     __shared__ float mm[W * 8], ml[W * 8];
     __shared__ float mo[W * 8 * D];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_wait();
+    pdl_launch_dependents();
     const int per_item = a.num_kv_heads * a.head_groups;
     const long long units = static_cast<long long>(*a.ws_count) * per_item;
     const int P = a.partition_size, B = a.block_size;
@@ -562,64 +601,146 @@ __global__ void __launch_bounds__(128) attend_f32_kernel(const DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// 3. reduce: merge the partitions of one (seq, head), in partition order
+// 3. reduce: merge the partitions of each multi-partition (seq, head)
 // ---------------------------------------------------------------------------
 
+// Contexts of at most REDUCE_HEADS_MAX_PARTS partitions: one warp per head
+// (4 heads of one sequence per CTA).  Lane i loads partition i's (max, sum);
+// the weights 2^(m_p - M) are shuffled to the lanes, which own float4 columns
+// of the output and sum the partitions in order.
+constexpr int REDUCE_HEADS_MAX_PARTS = 32;
+
 template <int D>
-__global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
-    constexpr int J = D / 32;
+__global__ void __launch_bounds__(128) reduce_heads_kernel(const DecodeArgs a) {
+    constexpr int C4 = D / 4, SUB = 32 / C4, U = 8;   // SUB lanes groups split the partitions
+    pdl_wait();
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quads = (a.num_heads + 3) / 4;
+    const int s = blockIdx.x / quads, head = (blockIdx.x - (blockIdx.x / quads) * quads) * 4 + warp;
+    const int ctx = clamp_context(a.context_lens[s], a.cap);
+    const int nparts = (ctx + a.partition_size - 1) / a.partition_size;
+    if (nparts <= 1 || head >= a.num_heads) return;   // single partitions are written by attend
+    const size_t row = static_cast<size_t>(s) * a.num_heads + head;
+    const float2 ml = lane < nparts ? a.ws_ml[row * a.max_parts + lane] : make_float2(NEG_INF, 0.f);
+    float M = ml.x;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
+    const float e = (lane < nparts && M != NEG_INF) ? exp2_approx(ml.x - M) : 0.f;
+    float L = e * ml.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(FULL_MASK, L, off);
+    const int c4 = lane % C4, sub = lane / C4;
+    const float4* accp = reinterpret_cast<const float4*>(a.ws_acc + row * a.max_parts * D) + c4;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < nparts; p0 += SUB * U) {
+        float4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int p = p0 + u * SUB + sub;
+            if (p < nparts) v[u] = accp[static_cast<size_t>(p) * C4];
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int p = p0 + u * SUB + sub;
+            const float w = __shfl_sync(FULL_MASK, e, p & 31);
+            if (p < nparts) {
+                o.x = fmaf(w, v[u].x, o.x);
+                o.y = fmaf(w, v[u].y, o.y);
+                o.z = fmaf(w, v[u].z, o.z);
+                o.w = fmaf(w, v[u].w, o.w);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = C4; off < 32; off <<= 1) {   // fold the partition groups, fixed order
+        o.x += __shfl_xor_sync(FULL_MASK, o.x, off);
+        o.y += __shfl_xor_sync(FULL_MASK, o.y, off);
+        o.z += __shfl_xor_sync(FULL_MASK, o.z, off);
+        o.w += __shfl_xor_sync(FULL_MASK, o.w, off);
+    }
+    if (sub == 0) {
+        const float r[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float val = L > 0.f ? r[k] / L : 0.f;
+            if (a.out_f32)
+                static_cast<float*>(a.out)[row * D + 4 * c4 + k] = val;
+            else
+                static_cast<__nv_bfloat16*>(a.out)[row * D + 4 * c4 + k] = __float2bfloat16_rn(val);
+        }
+    }
+}
+
+// Longer contexts: one CTA per (seq, head).  The 128 threads are D/4 float4
+// columns x G partition groups (group g takes partitions g, g+G, ...); the
+// groups are combined in a fixed order.
+template <int D>
+__global__ void __launch_bounds__(128) reduce_parts_kernel(const DecodeArgs a) {
+    constexpr int C4 = D / 4, G = 128 / C4, U = 8;
     __shared__ float red[4];
-    __shared__ float so[4][D];
-    __shared__ float sl[4];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __shared__ float4 so[G][C4];
+    __shared__ float sl[G];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x;
     const int s = blockIdx.x / a.num_heads, head = blockIdx.x - (blockIdx.x / a.num_heads) * a.num_heads;
     const int ctx = clamp_context(a.context_lens[s], a.cap);
-    const int P = a.partition_size;
-    const int nparts = (ctx + P - 1) / P;
-    if (nparts == 1) return;   // written directly by the attend kernel
+    const int nparts = (ctx + a.partition_size - 1) / a.partition_size;
+    if (nparts <= 1) return;   // written by the attend kernel
     const size_t row = static_cast<size_t>(s) * a.num_heads + head;
-    if (nparts == 0) {
-        for (int d = tid; d < D; d += 128) {
-            if (a.out_f32)
-                static_cast<float*>(a.out)[row * D + d] = 0.f;
-            else
-                static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(0.f);
-        }
-        return;
-    }
     const float2* mlp = a.ws_ml + row * a.max_parts;
-    const float* accp = a.ws_acc + row * a.max_parts * D;
+    const float4* accp = reinterpret_cast<const float4*>(a.ws_acc + row * a.max_parts * D);
     float M = NEG_INF;
     for (int p = tid; p < nparts; p += 128) M = fmaxf(M, mlp[p].x);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
-    if (lane == 0) red[warp] = M;
+    if ((tid & 31) == 0) red[tid >> 5] = M;
     __syncthreads();
     M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    float L = 0.f, o[J];
-#pragma unroll
-    for (int j = 0; j < J; ++j) o[j] = 0.f;
+    const int c4 = tid % C4, g = tid / C4;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = 0.f;
     if (M != NEG_INF) {
-        for (int p = warp; p < nparts; p += 4) {
-            const float2 v = mlp[p];
-            const float e = exp2_approx(v.x - M);
-            L += e * v.y;
+        for (int p0 = g; p0 < nparts; p0 += G * U) {
+            float4 v[U];
+            float2 ml[U];
 #pragma unroll
-            for (int j = 0; j < J; ++j) o[j] = fmaf(e, accp[static_cast<size_t>(p) * D + lane + 32 * j], o[j]);
+            for (int u = 0; u < U; ++u) {
+                const int p = p0 + u * G;
+                if (p < nparts) {
+                    ml[u] = mlp[p];
+                    v[u] = accp[static_cast<size_t>(p) * C4 + c4];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (p0 + u * G < nparts) {
+                    const float e = exp2_approx(ml[u].x - M);
+                    L = fmaf(e, ml[u].y, L);
+                    o.x = fmaf(e, v[u].x, o.x);
+                    o.y = fmaf(e, v[u].y, o.y);
+                    o.z = fmaf(e, v[u].z, o.z);
+                    o.w = fmaf(e, v[u].w, o.w);
+                }
+            }
         }
     }
-#pragma unroll
-    for (int j = 0; j < J; ++j) so[warp][lane + 32 * j] = o[j];
-    if (lane == 0) sl[warp] = L;
+    so[g][c4] = o;
+    if (c4 == 0) sl[g] = L;
     __syncthreads();
-    const float Lt = (sl[0] + sl[1]) + (sl[2] + sl[3]);
     for (int d = tid; d < D; d += 128) {
-        const float O = (so[0][d] + so[1][d]) + (so[2][d] + so[3][d]);
-        const float v = Lt > 0.f ? O / Lt : 0.f;
+        float O = 0.f, Lt = 0.f;
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+            O += reinterpret_cast<const float*>(&so[k][0])[d];
+            Lt += sl[k];
+        }
+        const float val = Lt > 0.f ? O / Lt : 0.f;
         if (a.out_f32)
-            static_cast<float*>(a.out)[row * D + d] = v;
+            static_cast<float*>(a.out)[row * D + d] = val;
         else
-            static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(v);
+            static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(val);
     }
 }
 
@@ -627,8 +748,14 @@ __global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
 // host side
 // ---------------------------------------------------------------------------
 
-constexpr int ATTEND_WARPS = 4;
-constexpr int ATTEND_STAGES = 3;
+#ifndef PA_ATTEND_WARPS
+#define PA_ATTEND_WARPS 3
+#endif
+#ifndef PA_ATTEND_STAGES
+#define PA_ATTEND_STAGES 2
+#endif
+constexpr int ATTEND_WARPS = PA_ATTEND_WARPS;    // warps per CTA of the bf16 attend kernel
+constexpr int ATTEND_STAGES = PA_ATTEND_STAGES;  // ring stages per warp
 
 inline size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
@@ -712,8 +839,7 @@ int launch_attend_bf16(const DecodeArgs& a, cudaStream_t st, long long unit_boun
     const long long cap_ctas = static_cast<long long>(per_sm) * sms;
     const int grid = static_cast<int>(unit_bound < cap_ctas ? unit_bound : cap_ctas);
     if (grid <= 0) return PA_OK;
-    kern<<<grid, W * 32, smem, st>>>(tk, tv, a);
-    return launch_status();
+    return launch_status(launch_pdl(kern, dim3(grid), dim3(W * 32), smem, st, tk, tv, a));
 }
 
 template <int D>
@@ -726,8 +852,7 @@ int launch_attend_f32(const DecodeArgs& a, cudaStream_t st, long long unit_bound
     const long long cap_ctas = static_cast<long long>(per_sm) * sms;
     const int grid = static_cast<int>(unit_bound < cap_ctas ? unit_bound : cap_ctas);
     if (grid <= 0) return PA_OK;
-    kern<<<grid, 128, 0, st>>>(a);
-    return launch_status();
+    return launch_status(launch_pdl(kern, dim3(grid), dim3(128), 0, st, a));
 }
 
 }  // namespace pa
@@ -816,8 +941,8 @@ extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, co
     const cudaStream_t st = as_stream(stream);
 
     if (phases & PA_PHASE_PLAN) {
-        plan_kernel<<<1, PLAN_THREADS, 0, st>>>(a);
-        if (launch_status() != PA_OK) return PA_ERR_CUDA;
+        if (launch_status(launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, st, a)) != PA_OK)
+            return PA_ERR_CUDA;
     }
     if (phases & PA_PHASE_ATTEND) {
         const long long unit_bound =
@@ -839,14 +964,20 @@ extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, co
         }
         if (rc != PA_OK) return rc;
     }
-    if (phases & PA_PHASE_REDUCE) {
-        const long long rows = static_cast<long long>(num_seqs) * num_heads;
-        if (rows > INT_MAX) return PA_ERR_UNSUPPORTED;
-        if (head_dim == 128)
-            reduce_kernel<128><<<static_cast<int>(rows), 128, 0, st>>>(a);
-        else
-            reduce_kernel<64><<<static_cast<int>(rows), 128, 0, st>>>(a);
-        if (launch_status() != PA_OK) return PA_ERR_CUDA;
+    if ((phases & PA_PHASE_REDUCE) && max_parts > 1) {
+        cudaError_t e;
+        if (max_parts <= REDUCE_HEADS_MAX_PARTS) {
+            const long long ctas = static_cast<long long>(num_seqs) * ((num_heads + 3) / 4);
+            if (ctas > INT_MAX) return PA_ERR_UNSUPPORTED;
+            e = head_dim == 128 ? launch_pdl(reduce_heads_kernel<128>, dim3(ctas), dim3(128), 0, st, a)
+                                : launch_pdl(reduce_heads_kernel<64>, dim3(ctas), dim3(128), 0, st, a);
+        } else {
+            const long long rows = static_cast<long long>(num_seqs) * num_heads;
+            if (rows > INT_MAX) return PA_ERR_UNSUPPORTED;
+            e = head_dim == 128 ? launch_pdl(reduce_parts_kernel<128>, dim3(rows), dim3(128), 0, st, a)
+                                : launch_pdl(reduce_parts_kernel<64>, dim3(rows), dim3(128), 0, st, a);
+        }
+        if (launch_status(e) != PA_OK) return PA_ERR_CUDA;
     }
     return PA_OK;
 }

@@ -32,6 +32,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// ---- programmatic dependent launch -----------------------------------------
+
+// Waits until the kernel this one depends on (the previous one in the stream)
+// has completed and its memory is visible; a no-op when launched normally.
+// Every CTA calls it before its first access to global memory.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel in the stream begin launching (its CTAs then wait in
+// pdl_wait until this grid completes).
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- mbarrier --------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

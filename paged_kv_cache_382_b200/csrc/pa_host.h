@@ -4,9 +4,11 @@
 
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 
 #include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "../../include/pa.h"
 
@@ -53,22 +55,52 @@ inline int prepare_kernel(KernelSlot& slot, const void* func, int threads, int s
         int c = slot.ctas_per_sm[dev].load(std::memory_order_relaxed);
         if (c > 0) return c;
     }
-    if (smem_bytes > 48 * 1024) {
-        if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
-            cudaSuccess)
-            return -1;
-    }
+    cudaError_t e = cudaSuccess;
+    if (smem_bytes > 48 * 1024)
+        e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     int c = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c, func, threads, smem_bytes) != cudaSuccess ||
-        c <= 0)
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c, func, threads, smem_bytes);
+    if (e != cudaSuccess || c <= 0) {
+#ifdef PA_DEBUG_ERRORS
+        fprintf(stderr, "libpa: kernel set-up failed (%d: %s), %d CTAs/SM at %d B shared memory\n",
+                static_cast<int>(e), cudaGetErrorString(e), c, smem_bytes);
+#endif
         return -1;
+    }
     slot.ctas_per_sm[dev].store(c, std::memory_order_relaxed);
     slot.smem[dev].store(smem_bytes, std::memory_order_release);
     return c;
 }
 
-inline int launch_status() {
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+// Launches `kernel` on `st` with programmatic stream serialisation allowed: it
+// may start while the previous kernel of the stream is finishing (each of
+// libpa's kernels waits for its predecessor with griddepcontrol.wait first).
+template <typename... KernelArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KernelArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// PA_ERR_CUDA if `launched` (the result of a launch call) or the last launch
+// or runtime call of this thread failed; clears the runtime's last error.
+// Build with -DPA_DEBUG_ERRORS to have the CUDA error text printed to stderr.
+inline int launch_status(cudaError_t launched = cudaSuccess) {
+    const cudaError_t last = cudaGetLastError();
+    const cudaError_t e = launched != cudaSuccess ? launched : last;
+#ifdef PA_DEBUG_ERRORS
+    if (e != cudaSuccess) fprintf(stderr, "libpa: CUDA error %d: %s\n", static_cast<int>(e), cudaGetErrorString(e));
+#endif
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa

@@ -24,7 +24,8 @@ def pa():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(pa_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:PA_API\s+)?(?:int|size_t|const char\*)\s+(pa_\w+)\s*\(", text,
+                                 flags=re.M)))
 
 
 def test_header_declares_the_boundary():
@@ -41,6 +42,14 @@ def test_library_exports_every_declared_symbol(pa):
     assert set(declared_functions()) <= set(pa.SIGNATURES)
 
 
+def test_library_exports_only_the_c_abi(pa):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.split() and line.split()[-2] in "TWVuBD"}
+    assert exported == set(declared_functions()), sorted(exported ^ set(declared_functions()))
+
+
 def test_status_strings_and_version(pa):
     assert pa.lib.pa_status_string(0).decode() == "PA_OK"
     assert b"workspace" in pa.lib.pa_status_string(3)
@@ -54,8 +63,9 @@ def test_workspace_bytes(pa):
     # several partitions: + (max, sum) and the fp32 partial outputs
     S, H, D, cap, P = 8, 64, 128, 131072, 512
     parts = cap // P
-    expect = 256 + (S * parts * 4 + 255) // 256 * 256 + (S * H * parts * 8 + 255) // 256 * 256 \
-        + (S * H * parts * D * 4 + 255) // 256 * 256
+    r = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    # header, work list, (max, sum), partial outputs
+    expect = 256 + r(S * parts * 4) + r(S * H * parts * 8) + r(S * H * parts * D * 4)
     assert ws(S, H, D, cap, P) == expect
     assert ws(-1, 1, 64, 10, 512) == 0
     assert ws(1, 1, 64, 10, 0) == 0
