@@ -23,6 +23,7 @@ from .paged_attention import (  # noqa: F401
     gather_kv,
     decode_attention,
     decode_attention_one,
+    prefill_attention,
     reshape_and_cache,
     copy_blocks,
 )

@@ -126,3 +126,33 @@ def copy_blocks(k_cache, v_cache, src_dst_pairs):
         k_out[int(dst)] = k_cache[int(src)]
         v_out[int(dst)] = v_cache[int(src)]
     return k_out, v_out
+
+
+def prefill_attention(q, k_cache, v_cache, block_tables, context_lens, query_start, scale):
+    """Causal attention of a chunk of new tokens against the paged context.
+
+    Sequence s holds context_lens[s] tokens; its last n_s = query_start[s+1] -
+    query_start[s] tokens are the new ones, whose queries are rows
+    query_start[s] .. query_start[s+1]-1 of q ([T][Hq][d]).  New token i of s sits
+    at position pos = context_lens[s] - n_s + i and attends to the tokens at
+    positions 0 .. pos of its own sequence (the prefill step of the
+    "PagedAttention blog", section 3(3), over K/V read through the block table).
+    Returns out [T][Hq][d] in fp64.
+    """
+    T, num_heads, head_dim = q.shape
+    num_kv_heads = k_cache.shape[1]
+    group = num_heads // num_kv_heads
+    out = np.zeros((T, num_heads, head_dim), dtype=np.float64)
+    for s in range(len(context_lens)):
+        ctx = int(context_lens[s])
+        first, last = int(query_start[s]), int(query_start[s + 1])
+        n_new = last - first
+        for kvh in range(num_kv_heads):
+            k_rows = gather_kv(k_cache, block_tables[s], ctx, kvh)
+            v_rows = gather_kv(v_cache, block_tables[s], ctx, kvh)
+            for i in range(n_new):
+                pos = ctx - n_new + i
+                for h in range(kvh * group, (kvh + 1) * group):
+                    out[first + i, h] = decode_attention_one(q[first + i, h], k_rows[: pos + 1],
+                                                             v_rows[: pos + 1], scale)
+    return out

@@ -508,3 +508,80 @@ def test_copy_mutants_are_caught(kind):
     except Exception:
         ok = False
     assert not ok
+
+
+# --------------------------------------------------------------------------
+# prefill (a chunk of new tokens, causal) against the paged context
+# --------------------------------------------------------------------------
+
+def prefill_problem(rng, ctx_lens, new_lens, Hq, Hkv, d, B):
+    p = random_problem(rng, ctx_lens, Hq, Hkv, d, B)
+    qs = np.concatenate([[0], np.cumsum(new_lens)]).astype(np.int64)
+    p["q"] = rng.standard_normal((int(qs[-1]), Hq, d))
+    p["query_start"] = qs
+    return p
+
+
+def pin_prefill_sdpa(prefill):
+    """torch SDPA in fp64 with an explicit mask: new token i of a sequence with
+    ctx tokens sees positions <= ctx - n + i."""
+    rng = np.random.default_rng(12)
+    ok = True
+    for ctx, new, Hq, Hkv, d, B in [([7, 33, 100], [3, 33, 1], 4, 4, 16, 4), ([50, 17], [20, 5], 8, 2, 32, 16)]:
+        p = prefill_problem(rng, ctx, new, Hq, Hkv, d, B)
+        got = prefill(p["q"], p["k_cache"], p["v_cache"], p["tables"], p["ctx"], p["query_start"], p["scale"])
+        for s, (c, n) in enumerate(zip(ctx, new)):
+            first = int(p["query_start"][s])
+            qt = torch.from_numpy(p["q"][first:first + n].transpose(1, 0, 2).copy())[None]   # [1][Hq][n][d]
+            kt = torch.from_numpy(p["k_seqs"][s])[None]
+            vt = torch.from_numpy(p["v_seqs"][s])[None]
+            pos = torch.arange(c - n, c)[:, None]
+            mask = torch.arange(c)[None, :] <= pos                                            # [n][c]
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qt, kt, vt, attn_mask=mask, scale=float(np.float32(p["scale"])), enable_gqa=(Hq != Hkv))
+            ref = ref[0].numpy().transpose(1, 0, 2)
+            ok &= float(np.abs(got[first:first + n] - ref).max()) <= 1e-12
+    return ok
+
+
+def pin_prefill_last_token_is_decode(prefill):
+    """The last new token of every sequence sees the whole context: it equals decode."""
+    rng = np.random.default_rng(13)
+    p = prefill_problem(rng, [9, 40, 3], [4, 1, 3], 4, 2, 16, 8)
+    got = prefill(p["q"], p["k_cache"], p["v_cache"], p["tables"], p["ctx"], p["query_start"], p["scale"])
+    last = p["query_start"][1:] - 1
+    dec = oracle.decode_attention(p["q"][last], p["k_cache"], p["v_cache"], p["tables"], p["ctx"], p["scale"])
+    return bool(np.array_equal(got[last], dec))
+
+
+def test_prefill_pins():
+    assert pin_prefill_sdpa(oracle.prefill_attention)
+    assert pin_prefill_last_token_is_decode(oracle.prefill_attention)
+
+
+def _mutant_prefill(kind):
+    def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale):
+        T, Hq, d = q.shape
+        Hkv = k_cache.shape[1]
+        g = Hq // Hkv
+        out = np.zeros((T, Hq, d))
+        for s in range(len(context_lens)):
+            ctx = int(context_lens[s])
+            first, last = int(query_start[s]), int(query_start[s + 1])
+            n = last - first
+            for kvh in range(Hkv):
+                K = oracle.gather_kv(k_cache, block_tables[s], ctx, kvh)
+                V = oracle.gather_kv(v_cache, block_tables[s], ctx, kvh)
+                for i in range(n):
+                    pos = {"no_causal_mask": ctx - 1, "positions_from_zero": i,
+                           "off_by_one": ctx - n + i - 1}.get(kind, ctx - n + i)
+                    for h in range(kvh * g, (kvh + 1) * g):
+                        out[first + i, h] = oracle.decode_attention_one(q[first + i, h], K[:pos + 1], V[:pos + 1],
+                                                                        scale)
+        return out
+    return prefill
+
+
+@pytest.mark.parametrize("kind", ["no_causal_mask", "positions_from_zero", "off_by_one"])
+def test_prefill_mutants_are_caught(kind):
+    assert not (pin_prefill_sdpa(_mutant_prefill(kind)) and pin_prefill_last_token_is_decode(_mutant_prefill(kind)))
