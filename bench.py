@@ -48,26 +48,26 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 CONFIGS = {
-    "llama7b": dict(builder="llama7b", kwargs={},
+    "llama7b": dict(max_len=2048, builder="llama7b", kwargs={},
                     desc="Llama-7B-like decode layer bf16: 64 seqs, 32 q = 32 kv heads, head_dim 128, "
                          "block_size 16, context lens uniform [128, 2048], 8192-block shuffled pool, "
                          "+ reshape_and_cache of 64 new tokens"),
-    "gqa": dict(builder="gqa", kwargs={},
+    "gqa": dict(max_len=8192, builder="gqa", kwargs={},
                 desc="GQA decode bf16: 256 seqs, 32 q / 8 kv heads, head_dim 128, block_size 16, "
                      "context lens log-normal (median 1000, sigma 1.0, capped 8192), 90% occupied pool"),
-    "shared_prefix": dict(builder="shared_prefix", kwargs=dict(prompt_len=512, suffix_max=512),
+    "shared_prefix": dict(max_len=1025, builder="shared_prefix", kwargs=dict(prompt_len=512, suffix_max=512),
                           desc="parallel sampling bf16: 16 prompts x 8 samples, 512-token prompt in "
                                "shared blocks, suffix uniform [0, 512], 32 q / 8 kv heads, head_dim 128"),
-    "shared_prefix_cow": dict(builder="shared_prefix", kwargs=dict(prompt_len=520, suffix_max=0),
+    "shared_prefix_cow": dict(max_len=521, builder="shared_prefix", kwargs=dict(prompt_len=520, suffix_max=0),
                               desc="parallel sampling bf16, first decode step after a 520-token prompt: "
                                    "112 copy-on-write block copies, 32 q / 8 kv heads, head_dim 128"),
-    "long_context_b8": dict(builder="long_context", kwargs=dict(block_size=8),
+    "long_context_b8": dict(max_len=131072, builder="long_context", kwargs=dict(block_size=8),
                             desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
                                  "64 q / 8 kv heads, head_dim 128, block_size 8, partitions of 512"),
-    "long_context_b16": dict(builder="long_context", kwargs=dict(block_size=16),
+    "long_context_b16": dict(max_len=131072, builder="long_context", kwargs=dict(block_size=16),
                              desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
                                   "64 q / 8 kv heads, head_dim 128, block_size 16, partitions of 512"),
-    "long_context_b32": dict(builder="long_context", kwargs=dict(block_size=32),
+    "long_context_b32": dict(max_len=131072, builder="long_context", kwargs=dict(block_size=32),
                              desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
                                   "64 q / 8 kv heads, head_dim 128, block_size 32, partitions of 512"),
 }
@@ -326,6 +326,16 @@ def nvsmi_id(local_index: int) -> str:
         return str(local_index)
 
 
+def kv_utilisation_summary(step, max_len):
+    """Tokens held / KV slots reserved for this batch: paged blocks against a
+    contiguous reservation of the workload's maximum length per sequence."""
+    from paged_kv_cache_382_b200.utilization import kv_utilisation
+
+    u = kv_utilisation(step.context_lens, step.block_size, max_len)
+    return {"paged": round(u["paged"], 4), "contiguous_max_len": round(u["contiguous"], 4),
+            "block_size": u["block_size"], "max_len": u["max_len"]}
+
+
 def build_step(config: str, seed: int, device, partition_size: int):
     from paged_kv_cache_382_b200 import workloads as W
 
@@ -473,6 +483,7 @@ def run_ours(args):
         "logical_bytes_per_step": logical_bytes,
         "effective_logical_gbs": round(logical_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
         "gpu_launches": ds.launches_per_step * K,
+        "kv_utilisation": kv_utilisation_summary(step, CONFIGS[args.config]["max_len"]),
         "roofline": {
             "kernel": "attend_bf16_kernel" if step.dtype == torch.bfloat16 else "attend_f32_kernel",
             "bound": "hbm",

@@ -173,6 +173,37 @@ PA_API int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const 
                      pa_dtype dtype, int32_t* dev_err, pa_stream stream, int phases);
 
 /*
+ * pa_prefill -- causal attention of a chunk of new tokens against the paged
+ * context (the prefill step of the "PagedAttention blog" section 3(3): the
+ * prompt's K/V are in the blocks, each new token attends to every token up to
+ * its own position).  Also serves chunked prefill and multi-token decode.
+ *
+ *   q, out        [num_tokens][num_heads][head_dim]: the new tokens of all sequences,
+ *                 sequence s owning rows query_start[s] .. query_start[s+1]-1
+ *   query_start   int32 [num_seqs + 1] (device), query_start[0] = 0,
+ *                 query_start[num_seqs] = num_tokens, non-decreasing
+ *   context_lens  int32 [num_seqs]: tokens of each sequence in the pool, its new tokens
+ *                 included (write them with pa_reshape_and_cache first); new token i of
+ *                 sequence s sits at position context_lens[s] - n_s + i
+ *   workspace     pa_prefill_workspace_bytes(num_tokens, num_heads, head_dim,
+ *                 max_context_len, partition_size) bytes, 256-byte aligned
+ * Other arguments, arithmetic and errors as for pa_decode (more new tokens than
+ * context: PA_DEVERR_CONTEXT, the excess positions see nothing).  Each new token
+ * is one query row of the decode kernels, with its context cut at its own
+ * position; consecutive new tokens of a sequence share every whole partition
+ * and are served together (up to 8 / group per K/V read).
+ */
+PA_API size_t pa_prefill_workspace_bytes(int num_tokens, int num_heads, int head_dim,
+                                         int max_context_len, int partition_size);
+PA_API int pa_prefill(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                      const int32_t* query_start, int num_seqs, int num_tokens, int num_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      int max_blocks_per_seq, int max_context_len, float scale, int partition_size,
+                      void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* dev_err,
+                      pa_stream stream);
+
+/*
  * pa_copy_blocks -- copy-on-write block copies ("PagedAttention blog" section 4,
  * step 2: the writer gets a new physical block holding a copy of the shared one).
  *

@@ -10,7 +10,10 @@
 //
 // How (three launches on the caller's stream):
 //   1. plan:    one CTA turns context_lens into a work list of (seq, partition)
-//               items, whole partitions first, ragged tails last.
+//               items, whole partitions first, ragged tails last.  Consecutive
+//               sequences whose block tables name the same physical blocks for
+//               a whole partition (parallel samples of one prompt) share one
+//               packed item: one K/V read serves all of them.
 //   2. attend:  persistent CTAs take (item, kv head, head group) units in a
 //               static stride.  One unit = one partition of up to
 //               partition_size tokens of one kv head, for the (up to 8) query
@@ -61,7 +64,7 @@ struct DecodeArgs {
     const int32_t* context_lens;
     int32_t* dev_err;
     int* ws_count;       // [1]   number of work items
-    int* ws_items;       // [num_seqs * max_parts]  item = seq * max_parts + partition
+    int* ws_items;       // [num_seqs * max_parts]  see make_item
     float2* ws_ml;       // [num_seqs][num_heads][max_parts]  (log2-domain max, sum)
     float* ws_acc;       // [num_seqs][num_heads][max_parts][head_dim]
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks;
@@ -72,7 +75,27 @@ struct DecodeArgs {
     int head_groups;     // ceil(group / 8): units per kv head
     float scale_log2;    // scale * log2(e)
     int out_f32;         // 1: out is fp32, 0: out is bf16
+    int pack;            // sequences a packed item may serve (8 / group; 1 = no packing)
+    const int32_t* row_seq;   // prefill: the sequence (block-table row) of each query row; null = identity
 };
+
+// Block-table row of query row s: its own row for decode; for prefill, the row
+// of the sequence the new token belongs to.
+__device__ __forceinline__ const int32_t* table_row(const DecodeArgs& a, int s) {
+    return a.block_tables + static_cast<size_t>(a.row_seq != nullptr ? a.row_seq[s] : s) * a.max_blocks;
+}
+
+// A work item names a partition p of sequence s and how many consecutive
+// sequences (s, s+1, ...) share that partition's blocks and are served by it.
+__host__ __device__ __forceinline__ int make_item(int s, int p, int count, int max_parts) {
+    return ((s * max_parts + p) << 3) | (count - 1);
+}
+__device__ __forceinline__ void split_item(int item, int max_parts, int& s, int& p, int& count) {
+    count = (item & 7) + 1;
+    const int sp = item >> 3;
+    s = sp / max_parts;
+    p = sp - s * max_parts;
+}
 
 __device__ __forceinline__ int clamp_context(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
 
@@ -111,55 +134,134 @@ __device__ int cta_exclusive_scan(int v, int* total, int* scratch) {
     return scratch[warp] + inc - v;
 }
 
+// Number of leading whole partitions that sequence s (context c) shares with
+// s + 1 (context c_next): the partitions whose block-table entries name the
+// same physical blocks.  first / first_next are the two tables' first entries
+// (loaded by the caller together with the context lengths, so a pair that
+// shares nothing costs no extra round trip); each compared partition costs one
+// round trip per 16 entries, all issued together.
+__device__ int shared_lead(const DecodeArgs& a, int s, int c, int c_next, int first, int first_next) {
+    const int P = a.partition_size, bpp = P / a.block_size;
+    const int kmax = min(c, c_next) / P;
+    if (a.pack <= 1 || kmax == 0 || first != first_next) return 0;
+    const int32_t* t0 = table_row(a, s);
+    const int32_t* t1 = table_row(a, s + 1);
+    if (t0 == t1) return kmax;   // two new tokens of one sequence (prefill)
+    int k = 0;
+    for (; k < kmax; ++k) {
+        bool same = true;
+        for (int i0 = 0; i0 < bpp; i0 += 16) {
+            int x[16], y[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (i0 + j < bpp) {
+                    x[j] = t0[k * bpp + i0 + j];
+                    y[j] = t1[k * bpp + i0 + j];
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (i0 + j < bpp) same &= x[j] == y[j];
+        }
+        if (!same) break;
+    }
+    return k;
+}
+
+// Whole-partition items of sequence s (context c), counted or written to out[].
+// Sequences are packed in aligned runs of a.pack: the first sequence of a run
+// emits one item per partition that its run-mates share with it (consecutive
+// links); a sequence not covered that way emits its own item.  `lead` holds
+// shared_lead of the sequences from lead_base on.
+template <bool WRITE>
+__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int* out) {
+    const int nfull = c / a.partition_size, m = a.pack;
+    if (m <= 1) {
+        if (WRITE)
+            for (int k = 0; k < nfull; ++k) out[k] = make_item(s, k, 1, a.max_parts);
+        return nfull;
+    }
+    const int c0 = s - s % m, j = s - c0;
+    int n = 0;
+    for (int k = 0; k < nfull; ++k) {
+        int cnt = 1;
+        while (cnt < m && c0 + cnt < a.num_seqs && lead[c0 + cnt - 1 - lead_base] > k) ++cnt;
+        if (j == 0 || j >= cnt) {
+            if (WRITE) out[n] = make_item(s, k, j == 0 ? cnt : 1, a.max_parts);
+            ++n;
+        }
+    }
+    return n;
+}
+
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
     __shared__ int scratch[33];
+    __shared__ int lead[PLAN_THREADS];
     pdl_wait();
     pdl_launch_dependents();
     const int P = a.partition_size;
-    // an item per whole partition, then one per ragged tail; an empty context
-    // is one item that writes zeros
-    auto counts = [&](int s, int& f, int& t) {
-        const int raw = a.context_lens[s];
-        const int c = clamp_context(raw, a.cap);
-        if (c != raw) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
-        f = c / P;
-        t = (c % P) != 0 || c == 0;
-    };
-    if (a.num_seqs <= PLAN_THREADS) {   // one pass
+    // Sequences are taken PLAN_THREADS at a time (a multiple of every packing
+    // run length).  Items: whole partitions first, then one per ragged tail,
+    // then one per empty context (it writes zeros).  One pass when the batch
+    // fits one chunk; otherwise a counting pass, then a writing pass.
+    const bool one_chunk = a.num_seqs <= PLAN_THREADS;
+    int full_total = 0, tail_total = 0;
+    int c = 0, f = 0, t = 0, ef = 0, et = 0;
+    for (int start = 0; start < a.num_seqs; start += PLAN_THREADS) {
+        const int s = start + threadIdx.x;
+        f = t = 0;
+        __syncthreads();
+        if (s < a.num_seqs) {
+            const bool has_next = s + 1 < a.num_seqs;
+            const int raw = a.context_lens[s];
+            const int raw_next = has_next ? a.context_lens[s + 1] : 0;
+            const int first = a.pack > 1 ? table_row(a, s)[0] : 0;
+            const int first_next = (a.pack > 1 && has_next) ? table_row(a, s + 1)[0] : 1;
+            c = clamp_context(raw, a.cap);
+            if (c != raw) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
+            lead[threadIdx.x] = shared_lead(a, s, c, clamp_context(raw_next, a.cap), first, first_next);
+            t = (c % P) != 0 || c == 0;
+        }
+        __syncthreads();
+        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, nullptr);
+        int cf = 0, ct = 0;
+        ef = cta_exclusive_scan(f, &cf, scratch);
+        et = cta_exclusive_scan(t, &ct, scratch);
+        full_total += cf;
+        tail_total += ct;
+    }
+    if (one_chunk) {
         const int s = threadIdx.x;
-        int f = 0, t = 0, full_total = 0, tail_total = 0;
-        if (s < a.num_seqs) counts(s, f, t);
-        const int ef = cta_exclusive_scan(f, &full_total, scratch);
-        const int et = cta_exclusive_scan(t, &tail_total, scratch);
-        for (int k = 0; k < f; ++k) a.ws_items[ef + k] = s * a.max_parts + k;
-        if (t) a.ws_items[full_total + et] = s * a.max_parts + f;
+        if (s < a.num_seqs) {
+            full_items<true>(a, s, c, lead, 0, a.ws_items + ef);
+            if (t) a.ws_items[full_total + et] = make_item(s, c / P, 1, a.max_parts);
+        }
         if (threadIdx.x == 0) *a.ws_count = full_total + tail_total;
         return;
     }
-    int nf = 0, nt = 0;
-    for (int s = threadIdx.x; s < a.num_seqs; s += PLAN_THREADS) {
-        int f, t;
-        counts(s, f, t);
-        nf += f;
-        nt += t;
-    }
-    int full_total = 0, tail_total = 0;
-    cta_exclusive_scan(nf, &full_total, scratch);
-    cta_exclusive_scan(nt, &tail_total, scratch);
     int base_full = 0, base_tail = full_total;
     for (int start = 0; start < a.num_seqs; start += PLAN_THREADS) {
         const int s = start + threadIdx.x;
-        int f = 0, t = 0;
+        f = t = 0;
+        __syncthreads();
         if (s < a.num_seqs) {
-            const int c = clamp_context(a.context_lens[s], a.cap);
-            f = c / P;
+            const bool has_next = s + 1 < a.num_seqs;
+            c = clamp_context(a.context_lens[s], a.cap);
+            const int c_next = has_next ? clamp_context(a.context_lens[s + 1], a.cap) : 0;
+            const int first = a.pack > 1 ? table_row(a, s)[0] : 0;
+            const int first_next = (a.pack > 1 && has_next) ? table_row(a, s + 1)[0] : 1;
+            lead[threadIdx.x] = shared_lead(a, s, c, c_next, first, first_next);
             t = (c % P) != 0 || c == 0;
         }
+        __syncthreads();
+        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, nullptr);
         int chunk_f = 0, chunk_t = 0;
-        const int ef = cta_exclusive_scan(f, &chunk_f, scratch);
-        const int et = cta_exclusive_scan(t, &chunk_t, scratch);
-        for (int k = 0; k < f; ++k) a.ws_items[base_full + ef + k] = s * a.max_parts + k;
-        if (t) a.ws_items[base_tail + et] = s * a.max_parts + f;
+        ef = cta_exclusive_scan(f, &chunk_f, scratch);
+        et = cta_exclusive_scan(t, &chunk_t, scratch);
+        if (s < a.num_seqs) {
+            full_items<true>(a, s, c, lead, start, a.ws_items + base_full + ef);
+            if (t) a.ws_items[base_tail + et] = make_item(s, c / P, 1, a.max_parts);
+        }
         base_full += chunk_f;
         base_tail += chunk_t;
     }
@@ -172,11 +274,31 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
 // mm, ml: [W][8] running max (log2 domain) and sum; mo: [W][8][D].
 // ---------------------------------------------------------------------------
 
+// Query row n (0..7, the mma N index) of a unit: the sequence (s + member)
+// and head it belongs to.  Up to 8 / group packed sequences x group heads, or
+// one sequence's heads head0 .. head0+7 when a kv head has more than 8.
+__device__ __forceinline__ void unit_row(const DecodeArgs& a, int kvh, int hg, int count, int n, int& member,
+                                         int& head, bool& valid) {
+    if (a.group <= 8) {
+        member = n / a.group;
+        head = kvh * a.group + (n - member * a.group);
+        valid = member < count;
+    } else {
+        member = 0;
+        head = kvh * a.group + hg * 8 + n;
+        valid = n < a.group - hg * 8;
+    }
+}
+
+__device__ __forceinline__ int unit_rows(const DecodeArgs& a, int hg, int count) {
+    return a.group <= 8 ? count * a.group : min(8, a.group - hg * 8);
+}
+
+// row_info[n] = (sequence, head, partitions of that sequence) of query row n.
 template <int W, int D>
 __device__ __forceinline__ void combine_store(const DecodeArgs& a, const float* mm, const float* ml,
-                                              const float* mo, int s, int p, int nparts, int head0,
-                                              int gsub) {
-    for (int idx = threadIdx.x; idx < gsub * D; idx += W * 32) {
+                                              const float* mo, const int3* row_info, int p, int nrows) {
+    for (int idx = threadIdx.x; idx < nrows * D; idx += W * 32) {
         const int n = idx / D, d = idx - (idx / D) * D;
         float M = NEG_INF;
 #pragma unroll
@@ -190,8 +312,9 @@ __device__ __forceinline__ void combine_store(const DecodeArgs& a, const float* 
                 O += e * mo[(w * 8 + n) * D + d];
             }
         }
-        const size_t row = static_cast<size_t>(s) * a.num_heads + head0 + n;
-        if (nparts <= 1) {
+        const int3 ri = row_info[n];
+        const size_t row = static_cast<size_t>(ri.x) * a.num_heads + ri.y;
+        if (ri.z <= 1) {
             const float v = L > 0.f ? O / L : 0.f;
             if (a.out_f32)
                 static_cast<float*>(a.out)[row * D + d] = v;
@@ -247,6 +370,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + W * NS * STAGE);
     int* tbl = reinterpret_cast<int*>(bars + W * NS);
     __shared__ int s_abort;
+    __shared__ int3 s_rows[8];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -290,22 +414,28 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int item = a.ws_items[u / per_item];
         const int r = static_cast<int>(u % per_item);
         const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
-        const int s = item / a.max_parts, p = item - (item / a.max_parts) * a.max_parts;
-        const int ctx = clamp_context(a.context_lens[s], a.cap);
+        int s, p, count;
+        split_item(item, a.max_parts, s, p, count);
+        const int ctx = clamp_context(a.context_lens[s], a.cap);   // packed items: whole partitions
         const int t0 = p * P;
         const int t1 = min(t0 + P, ctx);
         const int ntok = t1 - t0;
-        const int nparts = (ctx + P - 1) / P;
         const int nblk = ntok > 0 ? (t1 - 1) / B - t0 / B + 1 : 0;
-        const int gsub = min(8, a.group - hg * 8);
-        const int head0 = kvh * a.group + hg * 8;
+        const int nrows = unit_rows(a, hg, count);
 
         __syncthreads();   // the previous unit's epilogue is done with shared memory
         if (s_abort) break;
+        if (tid < 8) {
+            int member, head;
+            bool valid;
+            unit_row(a, kvh, hg, count, tid, member, head, valid);
+            const int cm = valid ? clamp_context(a.context_lens[s + member], a.cap) : 0;
+            s_rows[tid] = make_int3(s + member, head, (cm + P - 1) / P);
+        }
 
         // block-table slice of this partition, validated once
         int bad = 0;
-        const int32_t* trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks + t0 / B;
+        const int32_t* trow = table_row(a, s) + t0 / B;
         for (int i = tid; i < nblk; i += W * 32) {
             int b = trow[i];
             if (b < 0 || b >= a.num_blocks) {
@@ -314,12 +444,15 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             }
             tbl[i] = b;
         }
-        // q fragments (B operand of S^T = K Q^T): head g of the group, columns 16ks + 2c (+8)
+        // q fragments (B operand of S^T = K Q^T): query row g, columns 16ks + 2c (+8)
         uint32_t qf[KS][2];
-        if (g < gsub) {
+        int q_member, q_head;
+        bool q_valid;
+        unit_row(a, kvh, hg, count, g, q_member, q_head, q_valid);
+        if (q_valid) {
             const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
                 static_cast<const __nv_bfloat16*>(a.q) +
-                (static_cast<size_t>(s) * a.num_heads + head0 + g) * D);
+                (static_cast<size_t>(s + q_member) * a.num_heads + q_head) * D);
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 qf[ks][0] = qrow[8 * ks + c];
@@ -505,7 +638,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mo[(warp * 8 + 2 * c + 1) * D + 16 * i + 8 + g] = o[i][3];
         }
         __syncthreads();
-        combine_store<W, D>(a, mm, ml, mo, s, p, nparts, head0, gsub);
+        combine_store<W, D>(a, mm, ml, mo, s_rows, p, nrows);
         fence_proxy_async_smem();   // these generic accesses precede the next unit's bulk copies
     }
 }
@@ -519,6 +652,7 @@ __global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) 
     constexpr int W = 4, J = D / 32;
     __shared__ float mm[W * 8], ml[W * 8];
     __shared__ float mo[W * 8 * D];
+    __shared__ int3 s_rows[8];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_wait();
     pdl_launch_dependents();
@@ -533,7 +667,8 @@ __global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) 
         const int item = a.ws_items[u / per_item];
         const int r = static_cast<int>(u % per_item);
         const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
-        const int s = item / a.max_parts, p = item - (item / a.max_parts) * a.max_parts;
+        int s, p, count;
+        split_item(item, a.max_parts, s, p, count);   // this path is planned unpacked: count == 1
         const int ctx = clamp_context(a.context_lens[s], a.cap);
         const int t0 = p * P, t1 = min(t0 + P, ctx);
         const int nparts = (ctx + P - 1) / P;
@@ -553,7 +688,7 @@ __global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) 
             }
         }
         for (int t = t0 + warp; t < t1; t += W) {
-            const int phys = a.block_tables[static_cast<size_t>(s) * a.max_blocks + t / B];
+            const int phys = table_row(a, s)[t / B];
             if (phys < 0 || phys >= a.num_blocks) {
                 if (lane == 0) flag_error(a.dev_err, PA_DEVERR_BLOCK_ID);
                 continue;
@@ -584,6 +719,7 @@ __global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) 
             }
         }
         __syncthreads();   // the previous unit's epilogue is done with the merge buffers
+        if (tid < 8) s_rows[tid] = make_int3(s, head0 + tid, nparts);
         if (lane == 0) {
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
@@ -596,7 +732,7 @@ __global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) 
 #pragma unroll
             for (int j = 0; j < J; ++j) mo[(warp * 8 + n) * D + lane + 32 * j] = acc[n][j];
         __syncthreads();
-        combine_store<W, D>(a, mm, ml, mo, s, p, nparts, head0, gsub);
+        combine_store<W, D>(a, mm, ml, mo, s_rows, p, gsub);
     }
 }
 
@@ -745,6 +881,35 @@ __global__ void __launch_bounds__(128) reduce_parts_kernel(const DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// prefill: each new token becomes one query row of the decode machinery, with
+// its sequence's block table and a context that ends at its own position
+// (the causal mask), so consecutive new tokens of a sequence share every whole
+// partition and are served by packed units.
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256)
+prefill_rows_kernel(const int32_t* __restrict__ context_lens, const int32_t* __restrict__ query_start,
+                    int num_seqs, int num_tokens, int cap, int32_t* __restrict__ row_seq,
+                    int32_t* __restrict__ row_ctx, int32_t* dev_err) {
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < num_tokens; v += gridDim.x * blockDim.x) {
+        int lo = 0, hi = num_seqs - 1;   // the last sequence whose first new token is at or before v
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (query_start[mid] <= v) lo = mid; else hi = mid - 1;
+        }
+        const int first = query_start[lo], n_new = query_start[lo + 1] - first;
+        const int raw = context_lens[lo];
+        const int ctx = clamp_context(raw, cap);
+        const int pos = ctx - n_new + (v - first);
+        if (raw != ctx || n_new > ctx || v - first >= n_new || pos < 0) flag_error(dev_err, PA_DEVERR_CONTEXT);
+        row_seq[v] = lo;
+        row_ctx[v] = pos < 0 ? 0 : (pos + 1 > ctx ? ctx : pos + 1);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
@@ -866,13 +1031,17 @@ extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int hea
     return ws_layout(num_seqs, num_heads, head_dim, parts_for(max_context_len, partition_size)).total;
 }
 
-extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
-                                const void* v_cache, const int32_t* block_tables,
-                                const int32_t* context_lens, int num_seqs, int num_heads,
-                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                                int max_blocks_per_seq, int max_context_len, float scale,
-                                int partition_size, void* workspace, size_t workspace_bytes,
-                                pa_dtype dtype, int32_t* dev_err, pa_stream stream, int phases) {
+// Shared by decode and prefill; `row_seq` (device, may be null) maps each query
+// row to its block-table row.  `prep` (may be null) launches first, after the
+// validation, to produce row_seq / context_lens for prefill.
+template <typename Prep>
+static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                       const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                       int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                       int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                       int partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                       int32_t* dev_err, pa_stream stream, int phases, const int32_t* row_seq,
+                       Prep prep) {
     // ---- host-side validation: nothing is launched unless everything is sane
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0)
@@ -896,7 +1065,7 @@ extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, co
     long long cap = static_cast<long long>(max_blocks_per_seq) * block_size;
     if (max_context_len > 0 && max_context_len < cap) cap = max_context_len;
     const int max_parts = parts_for(static_cast<int>(cap), partition_size);
-    if (static_cast<long long>(num_seqs) * max_parts > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(num_seqs) * max_parts > INT_MAX / 16) return PA_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, max_parts);
     if (!workspace || !aligned_to(workspace, 256)) return PA_ERR_INVALID_ARG;
     if (workspace_bytes < L.total) return PA_ERR_WORKSPACE;
@@ -938,8 +1107,13 @@ extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, co
     a.head_groups = (a.group + 7) / 8;
     a.scale_log2 = scale * LOG2E;
     a.out_f32 = out_dtype == PA_F32;
+    a.row_seq = row_seq;
+    // bf16 units hold 8 query columns: up to 8 / group sequences sharing a
+    // partition's blocks can share one unit (fp32 units are never packed)
+    a.pack = (dtype == PA_BF16 && a.group <= 4) ? 8 / a.group : 1;
     const cudaStream_t st = as_stream(stream);
 
+    if (prep(st, a.cap) != PA_OK) return PA_ERR_CUDA;
     if (phases & PA_PHASE_PLAN) {
         if (launch_status(launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, st, a)) != PA_OK)
             return PA_ERR_CUDA;
@@ -980,6 +1154,63 @@ extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, co
         if (launch_status(e) != PA_OK) return PA_ERR_CUDA;
     }
     return PA_OK;
+}
+
+struct NoPrep {
+    int operator()(cudaStream_t, int) const { return PA_OK; }
+};
+
+extern "C" int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, int num_seqs, int num_heads,
+                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                int max_blocks_per_seq, int max_context_len, float scale,
+                                int partition_size, void* workspace, size_t workspace_bytes,
+                                pa_dtype dtype, int32_t* dev_err, pa_stream stream, int phases) {
+    return decode_impl(out, out_dtype, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, scale, partition_size, workspace, workspace_bytes, dtype, dev_err,
+                       stream, phases, nullptr, NoPrep());
+}
+
+static size_t prefill_rows_bytes(int num_tokens) {
+    return 2 * round_up(static_cast<size_t>(num_tokens) * sizeof(int32_t), 256);
+}
+
+extern "C" size_t pa_prefill_workspace_bytes(int num_tokens, int num_heads, int head_dim,
+                                             int max_context_len, int partition_size) {
+    const size_t d = pa_decode_workspace_bytes(num_tokens, num_heads, head_dim, max_context_len,
+                                               partition_size);
+    return d == 0 ? 0 : prefill_rows_bytes(num_tokens) + d;
+}
+
+extern "C" int pa_prefill(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                          const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                          const int32_t* query_start, int num_seqs, int num_tokens, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                          int max_blocks_per_seq, int max_context_len, float scale, int partition_size,
+                          void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* dev_err,
+                          pa_stream stream) {
+    if (num_seqs < 0 || num_tokens < 0) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (num_seqs == 0 || !context_lens || !query_start || !workspace) return PA_ERR_INVALID_ARG;
+    if (!aligned_to(context_lens, 4) || !aligned_to(query_start, 4) || !aligned_to(workspace, 256))
+        return PA_ERR_INVALID_ARG;
+    const size_t rows = prefill_rows_bytes(num_tokens);
+    if (workspace_bytes < rows) return PA_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* row_seq = reinterpret_cast<int32_t*>(ws);
+    int32_t* row_ctx = reinterpret_cast<int32_t*>(ws + rows / 2);
+    auto prep = [=](cudaStream_t st, int cap) {
+        const int threads = 256;
+        const int ctas = (num_tokens + threads - 1) / threads < 1024 ? (num_tokens + threads - 1) / threads : 1024;
+        return launch_status(launch_pdl(prefill_rows_kernel, dim3(ctas), dim3(threads), 0, st, context_lens,
+                                        query_start, num_seqs, num_tokens, cap, row_seq, row_ctx, dev_err));
+    };
+    return decode_impl(out, out_dtype, q, k_cache, v_cache, block_tables, row_ctx, num_tokens, num_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, max_context_len,
+                       scale, partition_size, ws + rows, workspace_bytes - rows, dtype, dev_err, stream,
+                       PA_PHASE_ALL, row_seq, prep);
 }
 
 extern "C" int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,

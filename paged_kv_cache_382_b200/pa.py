@@ -35,6 +35,9 @@ SIGNATURES = {
     "pa_decode": (_i, _DECODE_ARGS),
     "pa_decode_phases": (_i, _DECODE_ARGS + [_i]),
     "pa_copy_blocks": (_i, [_vp, _vp, _i64p, _i, _sz, _i, _i32p, _vp]),
+    "pa_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "pa_prefill": (_i, [_vp, _i, _vp, _vp, _vp, _i32p, _i32p, _i32p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                        _i, _vp, _sz, _i, _i32p, _vp]),
     "pa_decode_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i32p, _i32p, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                _i, _i, _i32p, _vp]),
     "pa_status_string": (ctypes.c_char_p, [_i]),
@@ -167,6 +170,36 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), dtype_code(dt),
         _opt_err(dev_err), _stream_handle(stream), phases)
     _check(rc, "pa_decode")
+    return out
+
+
+def prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+            block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor, scale: float,
+            *, max_context_len: int = 0, partition_size: int = 512,
+            workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Causal attention of new tokens q [T][Hq][d] (sequence s owns rows
+    query_start[s]..query_start[s+1]-1) against the paged context; writes ``out``."""
+    NB, Hkv, B, d = k_cache.shape
+    T, Hq, dq = q.shape
+    S = context_lens.shape[0]
+    if dq != d or tuple(out.shape) != (T, Hq, d) or tuple(query_start.shape) != (S + 1,):
+        raise ValueError("q/out must be [num_tokens][num_heads][head_dim], query_start [num_seqs + 1]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S:
+        raise ValueError("block_tables must be [num_seqs][max_blocks]")
+    dt = k_cache.dtype
+    if workspace is None:
+        cap = decode_capacity(block_tables, B, max_context_len)
+        n = lib.pa_prefill_workspace_bytes(T, Hq, d, cap, partition_size)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    rc = lib.pa_prefill(
+        _dev(out, "out"), dtype_code(out.dtype), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt),
+        _dev(v_cache, "v_cache", dt), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), _dev(query_start, "query_start", torch.int32), S, T,
+        Hq, Hkv, d, B, NB, block_tables.shape[1], max_context_len, float(scale), partition_size,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), dtype_code(dt), _opt_err(dev_err),
+        _stream_handle(stream))
+    _check(rc, "pa_prefill")
     return out
 
 

@@ -260,7 +260,9 @@ def gqa(seed: int = 0, sigma: float = 1.0, device="cpu", poison=False,
 
 
 def shared_prefix(seed: int = 0, prompt_len: int = 512, suffix_max: int = 512, prompts: int = 16,
-                  samples: int = 8, device="cpu", poison=False, partition_size: int = 512) -> DecodeStep:
+                  samples: int = 8, device="cpu", poison=False, partition_size: int = 512,
+                  num_heads: int = 32, num_kv_heads: int = 8, head_dim: int = 128,
+                  block_size: int = 16) -> DecodeStep:
     """Parallel sampling: ``prompts`` prompts x ``samples`` samples sharing the prompt's
     blocks (ref count = samples), per-sample suffix uniform [0, suffix_max] in private
     blocks; 32 q / 8 kv heads, d 128, bf16, block 16.  A partial last prompt block is
@@ -268,15 +270,15 @@ def shared_prefix(seed: int = 0, prompt_len: int = 512, suffix_max: int = 512, p
     rng = np.random.default_rng(seed)
     groups = [(prompt_len, [int(x) for x in rng.integers(0, suffix_max, size=samples, endpoint=True)])
               for _ in range(prompts)]
-    B = 16
+    B = block_size
     per_seq = [prompt_len + max(sfx) + 1 for _, sfx in groups]
     worst = prompts * (-(-prompt_len // B)) + sum(samples * (-(-(max(sfx) + 2) // B) + 1)
                                                   for _, sfx in groups)
     num_blocks = int(math.ceil(worst / 0.9))
     order = np.random.default_rng(seed + 7919).permutation(num_blocks)
     del per_seq
-    return _build(f"shared_prefix_p{prompt_len}_bf16", dtype=torch.bfloat16, num_heads=32,
-                  num_kv_heads=8, head_dim=128, block_size=B, num_blocks=num_blocks,
+    return _build(f"shared_prefix_p{prompt_len}_bf16", dtype=torch.bfloat16, num_heads=num_heads,
+                  num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=B, num_blocks=num_blocks,
                   free_order=order, groups=groups, seed=seed, device=device, poison=poison,
                   partition_size=partition_size,
                   meta=dict(prompts=prompts, samples=samples, prompt_len=prompt_len,

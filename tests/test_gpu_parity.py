@@ -336,6 +336,44 @@ def test_deterministic_and_shared_tables(pa):
     assert torch.equal(a[0], a[1])
 
 
+def unshared_copy(step):
+    """The same batch with every sequence's blocks copied to private physical
+    blocks: identical contents, no shared block ids, hence no packed units."""
+    B = step.block_size
+    ids, tables = [], np.full_like(step.block_tables, -1)
+    for sq in range(step.num_seqs):
+        nb = -(-int(step.context_lens[sq]) // B)
+        tables[sq, :nb] = np.arange(len(ids), len(ids) + nb)
+        ids.extend(int(b) for b in step.block_tables[sq, :nb])
+    idx = torch.tensor(ids, dtype=torch.long, device=step.k_cache.device)
+    out = W.DecodeStep(**{**step.__dict__})
+    out.k_cache = step.k_cache.index_select(0, idx).contiguous()
+    out.v_cache = step.v_cache.index_select(0, idx).contiguous()
+    out.num_blocks = len(ids)
+    out.block_tables = tables
+    out.slot_mapping = np.full_like(step.slot_mapping, -1)   # pools are compared after the step's writes
+    out.copy_pairs = np.zeros((0, 2), dtype=np.int64)
+    return out
+
+
+@pytest.mark.parametrize("heads", [(32, 8), (16, 8), (8, 8)], ids=["g4", "g2", "g1"])
+def test_packed_shared_prefix_units_are_bit_identical(pa, heads):
+    """Samples that share a prompt's blocks are served by packed units; the
+    result equals, bit for bit, the same batch with private copies of the blocks
+    (and the oracle)."""
+    Hq, Hkv = heads
+    step = W.shared_prefix(prompt_len=96, suffix_max=50, prompts=3, samples=5, device="cuda",
+                           partition_size=32, num_heads=Hq, num_kv_heads=Hkv, head_dim=128, block_size=16)
+    out, kc, vc, err, _ = run_gpu(pa, step)
+    assert err == 0
+    after = W.DecodeStep(**{**step.__dict__})
+    after.k_cache, after.v_cache = kc, vc          # the pool after this step's copies and writes
+    plain = unshared_copy(after)
+    out2, *_ = run_gpu(pa, plain)
+    assert torch.equal(out, out2)
+    assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, f"packed {heads}")
+
+
 def test_single_token_context_returns_the_value_row(pa):
     step = to_device(W.independent("one", [1, 1, 1], dtype=torch.bfloat16, num_heads=8, num_kv_heads=2,
                                    head_dim=128, block_size=8, seed=2))
@@ -395,3 +433,46 @@ def test_context_above_capacity_is_clamped_and_flagged(pa):
     clamped.context_lens = np.minimum(step.context_lens, 64)
     ref = full_oracle(clamped)
     assert_close(f64(out), ref, torch.bfloat16, torch.float32, "clamped")
+
+
+# ---------------------------------------------------------------------------
+# prefill: a chunk of new tokens attends causally to the paged context
+# ---------------------------------------------------------------------------
+
+PREFILL_CASES = [
+    # (context lens, new tokens, Hq, Hkv, d, B, P)
+    ([7, 40, 100], [7, 3, 33], 4, 4, 64, 16, 32),
+    ([300, 1029, 64, 1], [300, 45, 64, 1], 32, 8, 128, 16, 128),
+    ([257, 600], [120, 600], 8, 8, 128, 8, 64),
+    ([90, 2049], [17, 31], 16, 2, 128, 32, 512),
+    ([513, 80], [9, 80], 64, 8, 64, 4, 32),
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=lambda c: f"h{c[2]}x{c[3]}_d{c[4]}_b{c[5]}_p{c[6]}")
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_prefill_matches_oracle(pa, case, dtype):
+    ctx, new, Hq, Hkv, d, B, P = case
+    step = to_device(W.independent("prefill", ctx, dtype=dtype, num_heads=Hq, num_kv_heads=Hkv, head_dim=d,
+                                   block_size=B, seed=sum(new), poison=False, partition_size=P))
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    T = sum(new)
+    q = torch.empty(T, Hq, d, dtype=torch.float32, device="cuda").normal_(generator=gen).to(dtype)
+    qs = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    out = torch.empty(T, Hq, d, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.prefill(out, q, step.k_cache, step.v_cache, torch.from_numpy(step.block_tables).cuda(),
+               torch.from_numpy(step.context_lens).cuda(), torch.from_numpy(qs).cuda(), step.scale,
+               partition_size=P, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref = oracle.prefill_attention(f64(q), f64(step.k_cache), f64(step.v_cache), step.block_tables,
+                                   step.context_lens, qs, step.scale)
+    assert_close(f64(out), ref, dtype, torch.float32, str(case))
+    # the last new token of each sequence sees its whole context: it is the decode result
+    last = torch.from_numpy(qs[1:] - 1).long().cuda()
+    dec = torch.empty(len(ctx), Hq, d, dtype=torch.float32, device="cuda")
+    pa.decode(dec, q[last].contiguous(), step.k_cache, step.v_cache, torch.from_numpy(step.block_tables).cuda(),
+              torch.from_numpy(step.context_lens).cuda(), step.scale, partition_size=P)
+    torch.cuda.synchronize()
+    assert torch.equal(out[last], dec)
