@@ -71,6 +71,14 @@ CONFIGS = {
                              desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
                                   "64 q / 8 kv heads, head_dim 128, block_size 32, partitions of 512"),
 }
+CONFIGS["prefill_chunk"] = dict(
+    max_len=1280, builder="prefill_chunk", kwargs={},
+    desc="chunked prefill bf16: 16 seqs x (1024 cached + 256 new tokens), causal, 32 q / 8 kv heads, "
+         "head_dim 128, block_size 16, + reshape_and_cache of the 4096 new tokens")
+CONFIGS["host_block_manager"] = dict(
+    max_len=0, builder=None, kwargs={},
+    desc="host block manager (pa_bm_*, C++): 256 requests with a 512-token shared system prompt + "
+         "64 user tokens, then 256 decode steps of one token each, block_size 16")
 DEFAULT_CONFIG = "llama7b"
 ATTEND_SOURCES = ["paged_kv_cache_382_b200/csrc/decode.cu", "paged_kv_cache_382_b200/csrc/pa_device.cuh"]
 
@@ -292,7 +300,14 @@ class DeviceStep:
         self.ws = pa.alloc_workspace(step.num_seqs, step.num_heads, step.head_dim, self.cap, partition_size,
                                      dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.launches_per_step = (1 if len(step.copy_pairs) else 0) + 1 + 3
+        self.prefill = step.query_start is not None
+        if self.prefill:
+            T = step.q.shape[0]
+            self.qs = torch.from_numpy(step.query_start.astype(np.int32)).to(dev)
+            self.out = torch.empty(T, step.num_heads, step.head_dim, dtype=step.dtype, device=dev)
+            n = pa.lib.pa_prefill_workspace_bytes(T, step.num_heads, step.head_dim, self.cap, partition_size)
+            self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.launches_per_step = (1 if len(step.copy_pairs) else 0) + 1 + (4 if self.prefill else 3)
 
     def run(self, ev_attend=None, q=None, new_key=None, new_value=None, slots=None, tables=None, ctx=None,
             out=None):
@@ -306,6 +321,13 @@ class DeviceStep:
                 tables if tables is not None else self.tables, ctx if ctx is not None else self.ctx,
                 self.step.scale)
         kw = dict(max_context_len=self.cap, partition_size=self.P, workspace=self.ws, dev_err=self.err)
+        if self.prefill:
+            if ev_attend is not None:
+                ev_attend[0].record()
+            pa.prefill(*args[:6], self.qs, self.step.scale, **kw)
+            if ev_attend is not None:
+                ev_attend[1].record()
+            return
         pa.decode(*args, phases=pa.PHASE_PLAN, **kw)
         if ev_attend is not None:
             ev_attend[0].record()
@@ -408,6 +430,11 @@ def run_ours(args):
     ds = DeviceStep(pa, step, args.partition_size)
     alg_bytes = W.algorithmic_bytes(step, unique=True)
     logical_bytes = W.algorithmic_bytes(step, unique=False)
+    if ds.prefill:   # q and out hold every new token
+        extra = 2 * (step.q.shape[0] - step.num_seqs) * step.num_heads * step.head_dim * step.element_bytes
+        alg_bytes += extra
+        logical_bytes += extra
+        args.no_e2e = True
     ctx_tokens = int(step.context_lens.sum())
 
     stream = torch.cuda.current_stream()
@@ -448,9 +475,14 @@ def run_ours(args):
 
     cpu = None
     if pool is not None:
-        cpu = cpu_baseline(step, pool, cores, args.cpu_core_seconds)
+        if not ds.prefill:
+            cpu = cpu_baseline(step, pool, cores, args.cpu_core_seconds)
         pool.close()
     if rank != 0:
+        return
+    if ds.prefill:
+        print(json.dumps(prefill_line(args, step, world, K, max_ms, attend_ms, alg_bytes, clock_info, ds)),
+              flush=True)
         return
     traffic = profiled_traffic(args.config)
     line = {
@@ -506,6 +538,42 @@ def run_ours(args):
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": round(e2e_ms / e2e["steps"], 5), "steps": e2e["steps"]}
     print(json.dumps(line), flush=True)
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured sustained cuBLAS bf16"
+    except (OSError, KeyError, ValueError):
+        return 1400.0, "fallback sustained bf16"
+
+
+def prefill_line(args, step, world, K, max_ms, prefill_ms, alg_bytes, clock_info, ds):
+    """The chunked-prefill workload: useful attention FLOP/s against the tensor roofline."""
+    from paged_kv_cache_382_b200 import workloads as W
+
+    flops = W.prefill_flops(step)
+    peak, kind = measured_tensor_peak()
+    tflops_step = flops * K * world / (max_ms * 1e-3) / 1e12
+    tflops_call = flops / (prefill_ms * 1e-3) / 1e12
+    return {
+        "metric": "paged prefill attention TFLOP/s (causal, useful flops) and KV GB/s",
+        "value": round(tflops_step, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(max_ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; K/V/q ~ N(0,1) generated on the device by torch, no dataset)",
+        "config": {"workload": CONFIGS[args.config]["desc"], "name": args.config,
+                   "new_tokens_per_gpu": int(step.q.shape[0]), "partition_size": args.partition_size},
+        "kv_gbs": round(alg_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
+        "flops_per_step": flops,
+        "gpu_launches": ds.launches_per_step * K,
+        "roofline": {"kernel": "pa_prefill (rows, plan, attend, reduce)", "bound": "tensor",
+                     "achieved": round(tflops_call, 2), "peak": peak, "peak_kind": kind, "unit": "TFLOP/s",
+                     "frac": round(tflops_call / peak, 4), "traffic": None,
+                     "prefill_ms": round(prefill_ms, 5)},
+        "clocks": clock_info, "e2e": None, "cpu_baseline": None,
+    }
 
 
 def run_e2e(ds, step, alg_bytes, warmup, steps):
@@ -662,8 +730,55 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_block_manager(args):
+    """Tokens per second through the library's host block manager: prompt
+    admission with and without prefix caching, then single-token decode
+    appends (CPU only)."""
+    import numpy as np
+
+    from paged_kv_cache_382_b200 import build as _build
+
+    _build.build()
+    from paged_kv_cache_382_b200 import pa
+
+    rng = np.random.default_rng(args.seed)
+    R, P_SYS, USER, STEPS, B = 256, 512, 64, 256, 16
+    system = rng.integers(0, 32000, size=P_SYS).astype(np.int32)
+    prompts = [np.concatenate([system, rng.integers(0, 32000, size=USER).astype(np.int32)]) for _ in range(R)]
+    res = {}
+    for cache in (False, True):
+        m = pa.NativeBlockManager(R * ((P_SYS + USER + STEPS) // B + 2), B, prefix_cache=cache)
+        t0 = time.perf_counter()
+        cached = 0
+        for r in range(R):
+            m.add(r)
+            _, _, c = m.append(r, prompts[r] if cache else len(prompts[r]))
+            cached += c
+        t1 = time.perf_counter()
+        one = np.zeros(1, dtype=np.int32)
+        for _ in range(STEPS):
+            for r in range(R):
+                m.append(r, one if cache else 1)
+        t2 = time.perf_counter()
+        key = "prefix_cache" if cache else "no_cache"
+        res[key] = {"admit_tokens_per_s": round(R * (P_SYS + USER) / (t1 - t0), 1),
+                    "decode_appends_per_s": round(R * STEPS / (t2 - t1), 1),
+                    "cached_token_fraction": round(cached / (R * (P_SYS + USER)), 4),
+                    "blocks_in_use": R * ((P_SYS + USER + STEPS) // B + 2) - m.num_free}
+    line = {"metric": "host block manager tokens/s (admission and decode appends)",
+            "value": res["prefix_cache"]["admit_tokens_per_s"], "unit": "tokens/s", "n_gpus": 0,
+            "higher_is_better": True, "data": "synthetic token ids (seeded)",
+            "config": {"workload": CONFIGS["host_block_manager"]["desc"], "name": "host_block_manager"},
+            "results": res,
+            "note": "timed through the Python binding (ctypes call per request / per step)"}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.config == "host_block_manager":
+        run_block_manager(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

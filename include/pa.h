@@ -255,6 +255,60 @@ PA_API int pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* q, const
                       int max_blocks_per_seq, int max_context_len, float scale,
                       int partition_size, pa_dtype dtype, int32_t* dev_err, pa_stream stream);
 
+/*
+ * Host block manager -- the bookkeeping that produces block tables, slot
+ * mappings and copy-on-write pairs (host memory only; no CUDA call).  After
+ * "Month 2 · PagedAttention" sections 02-04 and the "PagedAttention blog"
+ * sections 3(3) and 4:
+ *  - a pool of num_blocks physical blocks of block_size slots, a free list
+ *    (initial order `free_order`, a permutation of 0..num_blocks-1, or NULL for
+ *    0, 1, 2, ...) and a reference count per block;
+ *  - a block is taken only when a sequence's token crosses into a new logical
+ *    block; forked sequences share blocks (counts raised); appending into a
+ *    shared partly filled block first moves the writer to a fresh block and
+ *    reports the (old, new) copy, the last sharer writes in place;
+ *  - freeing a sequence drops its counts, last block first; blocks at zero go
+ *    to the back of the free list;
+ *  - with enable_prefix_cache, every full block is keyed by a hash chained over
+ *    its token ids and its predecessor's key; when a sequence starts a new
+ *    logical block and the next block_size tokens match a cached block (key and
+ *    stored tokens), that block is referenced instead of allocated and its
+ *    tokens' slots are -1 (already in the pool: skip their K/V writes).  A
+ *    cached block stays cached while it sits in the free list and is evicted
+ *    (least recently freed first) when it is reused for other data.
+ * Not thread-safe per manager.  Sequences are named by caller-chosen ids.
+ */
+typedef struct pa_block_manager pa_block_manager;
+/* NULL on bad arguments (num_blocks or block_size <= 0, free_order not a permutation). */
+PA_API pa_block_manager* pa_bm_create(int num_blocks, int block_size, const int32_t* free_order,
+                                      int enable_prefix_cache);
+PA_API void pa_bm_destroy(pa_block_manager* manager);
+/* PA_ERR_INVALID_ARG if the id is in use. */
+PA_API int pa_bm_add_sequence(pa_block_manager* manager, int64_t seq_id);
+/* child shares every block of parent; PA_ERR_INVALID_ARG if parent is unknown or child in use. */
+PA_API int pa_bm_fork(pa_block_manager* manager, int64_t parent, int64_t child);
+PA_API int pa_bm_free(pa_block_manager* manager, int64_t seq_id);
+/*
+ * Appends num_tokens tokens to seq_id.  slots[num_tokens] receives each token's
+ * slot (block * block_size + offset, or -1 for a token found in the prefix
+ * cache); copies[2 * max_copies] receives the (src, dst) block copies that must
+ * run before the writes (may be NULL if max_copies is 0), *num_copies their
+ * number, *num_cached_tokens (nullable) the tokens served from the cache.
+ * token_ids[num_tokens] is required with prefix caching, else ignored.
+ * PA_ERR_WORKSPACE if the pool runs out of free blocks or more than max_copies
+ * copies are needed: the tokens before that point stay appended.
+ */
+PA_API int pa_bm_append(pa_block_manager* manager, int64_t seq_id, const int32_t* token_ids,
+                        int num_tokens, int64_t* slots, int64_t* copies, int max_copies,
+                        int* num_copies, int* num_cached_tokens);
+/* The sequence's block table (out may be NULL to query *num_blocks); PA_ERR_WORKSPACE if
+ * it has more than max_blocks entries.  *num_tokens (nullable) gets its length. */
+PA_API int pa_bm_block_table(const pa_block_manager* manager, int64_t seq_id, int32_t* out,
+                             int max_blocks, int* num_blocks, int64_t* num_tokens);
+PA_API int pa_bm_num_free(const pa_block_manager* manager);
+/* -1 for a bad block id. */
+PA_API int pa_bm_ref_count(const pa_block_manager* manager, int block);
+
 /* Human-readable name of a pa_status value (static storage). */
 PA_API const char* pa_status_string(int status);
 

@@ -130,7 +130,8 @@ class BlockManager:
         return Sequence(block_table=list(seq.block_table), num_tokens=seq.num_tokens)
 
     def free(self, seq: Sequence) -> None:
-        for block in seq.block_table:
+        # last block first: under least-recently-freed reuse a shared prefix stays longest
+        for block in reversed(seq.block_table):
             self.pool.decref(block)
         seq.block_table = []
         seq.num_tokens = 0

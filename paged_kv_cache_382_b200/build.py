@@ -2,7 +2,8 @@
 
     python -m paged_kv_cache_382_b200.build [--verbose]
 
-nvcc compiles every ``csrc/*.cu`` for ``sm_100a`` only and links one shared
+nvcc compiles every ``csrc/*.cu`` for ``sm_100a`` only (and the host-only
+``csrc/*.cpp``) and links one shared
 library next to this file; the CUDA runtime is linked statically, so the
 library needs nothing from the environment beyond the NVIDIA driver.
 """
@@ -18,7 +19,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB_PATH = os.path.join(HERE, "libpa.so")
-SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
+SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")) + glob.glob(os.path.join(HERE, "csrc", "*.cpp")))
 DEPS = SOURCES + [os.path.abspath(__file__)] + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")) +
                         glob.glob(os.path.join(HERE, "csrc", "*.h")) +
                         glob.glob(os.path.join(ROOT, "include", "*.h")))

@@ -40,6 +40,17 @@ SIGNATURES = {
                         _i, _vp, _sz, _i, _i32p, _vp]),
     "pa_decode_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i32p, _i32p, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                _i, _i, _i32p, _vp]),
+    "pa_bm_create": (ctypes.c_void_p, [_i, _i, _vp, _i]),
+    "pa_bm_destroy": (None, [_vp]),
+    "pa_bm_add_sequence": (_i, [_vp, ctypes.c_int64]),
+    "pa_bm_fork": (_i, [_vp, ctypes.c_int64, ctypes.c_int64]),
+    "pa_bm_free": (_i, [_vp, ctypes.c_int64]),
+    "pa_bm_append": (_i, [_vp, ctypes.c_int64, _vp, _i, _vp, _vp, _i, ctypes.POINTER(ctypes.c_int),
+                          ctypes.POINTER(ctypes.c_int)]),
+    "pa_bm_block_table": (_i, [_vp, ctypes.c_int64, _vp, _i, ctypes.POINTER(ctypes.c_int),
+                               ctypes.POINTER(ctypes.c_int64)]),
+    "pa_bm_num_free": (_i, [_vp]),
+    "pa_bm_ref_count": (_i, [_vp, _i]),
     "pa_status_string": (ctypes.c_char_p, [_i]),
     "pa_version": (_i, []),
 }
@@ -241,3 +252,80 @@ def decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_
         _stream_handle(stream))
     _check(rc, "pa_decode_noalloc")
     return out
+
+
+class NativeBlockManager:
+    """Handle on the library's host block manager (``pa_bm_*``): free list, ref
+    counts, lazy allocation, fork, copy-on-write planning and, optionally,
+    prefix caching by chained block keys.  Host memory only."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None, prefix_cache: bool = False):
+        import numpy as np
+
+        self._np = np
+        self.block_size = int(block_size)
+        order = None
+        if free_order is not None:
+            self._order = np.ascontiguousarray(free_order, dtype=np.int32)
+            order = self._order.ctypes.data
+        self._h = lib.pa_bm_create(int(num_blocks), int(block_size), order, int(bool(prefix_cache)))
+        if not self._h:
+            raise ValueError("pa_bm_create rejected its arguments")
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            lib.pa_bm_destroy(h)
+            self._h = None
+
+    def add(self, seq_id: int) -> None:
+        _check(lib.pa_bm_add_sequence(self._h, seq_id), "pa_bm_add_sequence")
+
+    def fork(self, parent: int, child: int) -> None:
+        _check(lib.pa_bm_fork(self._h, parent, child), "pa_bm_fork")
+
+    def free(self, seq_id: int) -> None:
+        _check(lib.pa_bm_free(self._h, seq_id), "pa_bm_free")
+
+    def append(self, seq_id: int, tokens):
+        """Append tokens (a count, or token ids when prefix caching).  Returns
+        (slots int64 array, [(src, dst) copies], tokens served from the cache)."""
+        np = self._np
+        ids = None
+        if isinstance(tokens, int):
+            n = tokens
+        else:
+            ids = np.ascontiguousarray(tokens, dtype=np.int32)
+            n = len(ids)
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        cap = max(n, 1)
+        copies = np.empty(2 * cap, dtype=np.int64)
+        ncopies, ncached = ctypes.c_int(0), ctypes.c_int(0)
+        rc = lib.pa_bm_append(self._h, seq_id, None if ids is None else ids.ctypes.data, n, slots.ctypes.data,
+                              copies.ctypes.data, cap, ctypes.byref(ncopies), ctypes.byref(ncached))
+        _check(rc, "pa_bm_append")
+        pairs = [(int(copies[2 * i]), int(copies[2 * i + 1])) for i in range(ncopies.value)]
+        return slots[:n], pairs, ncached.value
+
+    def block_table(self, seq_id: int):
+        np = self._np
+        nb, nt = ctypes.c_int(0), ctypes.c_int64(0)
+        rc = lib.pa_bm_block_table(self._h, seq_id, None, 0, ctypes.byref(nb), ctypes.byref(nt))
+        if rc not in (PA_OK, PA_ERR_WORKSPACE):
+            _check(rc, "pa_bm_block_table")
+        out = np.empty(max(nb.value, 1), dtype=np.int32)
+        _check(lib.pa_bm_block_table(self._h, seq_id, out.ctypes.data, len(out), ctypes.byref(nb),
+                                     ctypes.byref(nt)), "pa_bm_block_table")
+        return [int(b) for b in out[: nb.value]]
+
+    def num_tokens(self, seq_id: int) -> int:
+        nb, nt = ctypes.c_int(0), ctypes.c_int64(0)
+        lib.pa_bm_block_table(self._h, seq_id, None, 0, ctypes.byref(nb), ctypes.byref(nt))
+        return int(nt.value)
+
+    @property
+    def num_free(self) -> int:
+        return int(lib.pa_bm_num_free(self._h))
+
+    def ref_count(self, block: int) -> int:
+        return int(lib.pa_bm_ref_count(self._h, block))

@@ -60,6 +60,7 @@ class DecodeStep:
     slot_mapping: np.ndarray          # int64 [T]; -1 = no write
     copy_pairs: np.ndarray            # int64 [n][2] (src, dst)
     meta: Dict = field(default_factory=dict)
+    query_start: Optional[np.ndarray] = None   # prefill: int32 [S + 1]; q / new K,V hold every new token
 
     @property
     def num_seqs(self) -> int:
@@ -296,10 +297,60 @@ def long_context(seed: int = 0, block_size: int = 16, device="cpu", poison=False
                        seed=seed, device=device, poison=poison, partition_size=partition_size)
 
 
+def prefill_chunk(seed: int = 0, num_seqs: int = 16, cached: int = 1024, new: int = 256, device="cpu",
+                  num_heads: int = 32, num_kv_heads: int = 8, head_dim: int = 128, block_size: int = 16,
+                  partition_size: int = 512, dtype=torch.bfloat16) -> DecodeStep:
+    """Chunked prefill: each sequence holds ``cached`` tokens and appends ``new``
+    tokens whose K/V are written this step and whose queries attend causally."""
+    used = num_seqs * (-(-(cached + new) // block_size))
+    num_blocks = int(math.ceil(used / 0.9))
+    order = np.random.default_rng(seed + 7919).permutation(num_blocks)
+    pool = BlockPool(num_blocks, order)
+    mgr = BlockManager(pool, block_size)
+    seqs, slots = [], []
+    for _ in range(num_seqs):
+        sq = mgr.new_sequence()
+        mgr.append_tokens(sq, cached)
+        sl, _ = mgr.append_tokens(sq, new)
+        slots.extend(sl)
+        seqs.append(sq)
+    gen = _generator(device, seed)
+    Hkv, d, B = num_kv_heads, head_dim, block_size
+    k_cache = _normal((num_blocks, Hkv, B, d), dtype, device, gen)
+    v_cache = _normal((num_blocks, Hkv, B, d), dtype, device, gen)
+    T = num_seqs * new
+    q = _normal((T, num_heads, d), dtype, device, gen)
+    new_key = _normal((T, Hkv, d), dtype, device, gen)
+    new_value = _normal((T, Hkv, d), dtype, device, gen)
+    return DecodeStep(
+        name=f"prefill_{cached}+{new}", dtype=dtype, num_heads=num_heads, num_kv_heads=Hkv, head_dim=d,
+        block_size=B, num_blocks=num_blocks,
+        context_lens=np.array([sq.num_tokens for sq in seqs], dtype=np.int32),
+        block_tables=block_table_array(seqs), scale=float(np.float32(1.0 / math.sqrt(d))),
+        partition_size=partition_size, q=q, k_cache=k_cache, v_cache=v_cache, new_key=new_key,
+        new_value=new_value, slot_mapping=np.array(slots, dtype=np.int64),
+        copy_pairs=np.zeros((0, 2), dtype=np.int64), meta=dict(cached=cached, new=new),
+        query_start=np.arange(0, T + 1, new, dtype=np.int32))
+
+
+def prefill_flops(step: DecodeStep) -> int:
+    """Useful multiply-adds x 2 of a prefill step: q.K and p.V of every new token over
+    the positions it sees, 4 * d * Hq * (pos + 1) each."""
+    total = 0
+    qs = step.query_start
+    for s in range(step.num_seqs):
+        n = int(qs[s + 1] - qs[s])
+        c = int(step.context_lens[s])
+        # positions c-n .. c-1, each seeing pos + 1 tokens
+        total += sum(range(c - n + 1, c + 1))
+    return 4 * step.head_dim * step.num_heads * total
+
+
 WORKLOADS = {
     "tiny": tiny,
     "llama7b": llama7b,
     "gqa": gqa,
     "shared_prefix": shared_prefix,
     "long_context": long_context,
+    "prefill_chunk": prefill_chunk,
 }
