@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(HERE, "libpa.so")
 SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")) + glob.glob(os.path.join(HERE, "csrc", "*.cpp")))
 DEPS = SOURCES + [os.path.abspath(__file__)] + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")) +
                         glob.glob(os.path.join(HERE, "csrc", "*.h")) +
+                        glob.glob(os.path.join(HERE, "csrc", "*.map")) +
                         glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -48,6 +49,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = LIB_PATH + ".tmp"
     cmd = [nvcc_path(), "-O3", "-std=c++17", *ARCH_FLAGS, "-lineinfo",
            "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden", "-shared", "-I", os.path.join(ROOT, "include"),
+           "-Xlinker", "--version-script=" + os.path.join(HERE, "csrc", "libpa.map"),
            "-o", tmp, *SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")

@@ -24,8 +24,7 @@ def pa():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:PA_API\s+)?(?:int|size_t|const char\*)\s+(pa_\w+)\s*\(", text,
-                                 flags=re.M)))
+    return sorted(set(re.findall(r"^\s*PA_API\s+[\w\s\*]*?\b(pa_\w+)\s*\(", text, flags=re.M)))
 
 
 def test_header_declares_the_boundary():
