@@ -307,7 +307,12 @@ class DeviceStep:
             self.out = torch.empty(T, step.num_heads, step.head_dim, dtype=step.dtype, device=dev)
             n = pa.lib.pa_prefill_workspace_bytes(T, step.num_heads, step.head_dim, self.cap, partition_size)
             self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
-        self.launches_per_step = (1 if len(step.copy_pairs) else 0) + 1 + (4 if self.prefill else 3)
+        self.tensor_core_prefill = self.prefill and pa.prefill_uses_tensor_cores(
+            step.dtype, step.num_heads, step.num_kv_heads, step.head_dim, step.block_size)
+        # copy_blocks, reshape_and_cache, then plan/attend/reduce (decode), rows/plan/attend/reduce
+        # (prefill by decode rows) or plan/attend (tensor-core prefill)
+        body = 3 if not self.prefill else (2 if self.tensor_core_prefill else 4)
+        self.launches_per_step = (1 if len(step.copy_pairs) else 0) + 1 + body
 
     def run(self, ev_attend=None, q=None, new_key=None, new_value=None, slots=None, tables=None, ctx=None,
             out=None):
@@ -568,10 +573,13 @@ def prefill_line(args, step, world, K, max_ms, prefill_ms, alg_bytes, clock_info
         "kv_gbs": round(alg_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
         "flops_per_step": flops,
         "gpu_launches": ds.launches_per_step * K,
-        "roofline": {"kernel": "pa_prefill (rows, plan, attend, reduce)", "bound": "tensor",
+        "roofline": {"kernel": ("pa_prefill (tcgen05: plan, attend)" if ds.tensor_core_prefill
+                                else "pa_prefill (decode rows: rows, plan, attend, reduce)"),
+                     "bound": "tensor",
                      "achieved": round(tflops_call, 2), "peak": peak, "peak_kind": kind, "unit": "TFLOP/s",
                      "frac": round(tflops_call / peak, 4), "traffic": None,
-                     "prefill_ms": round(prefill_ms, 5)},
+                     "prefill_ms": round(prefill_ms, 5),
+                     "mma_flops_issued": (W.prefill_tc_mma_flops(step) if ds.tensor_core_prefill else None)},
         "clocks": clock_info, "e2e": None, "cpu_baseline": None,
     }
 

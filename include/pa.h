@@ -188,13 +188,26 @@ PA_API int pa_decode_phases(void* out, pa_dtype out_dtype, const void* q, const 
  *   workspace     pa_prefill_workspace_bytes(num_tokens, num_heads, head_dim,
  *                 max_context_len, partition_size) bytes, 256-byte aligned
  * Other arguments, arithmetic and errors as for pa_decode (more new tokens than
- * context: PA_DEVERR_CONTEXT, the excess positions see nothing).  Each new token
- * is one query row of the decode kernels, with its context cut at its own
- * position; consecutive new tokens of a sequence share every whole partition
- * and are served together (up to 8 / group per K/V read).
+ * context: PA_DEVERR_CONTEXT, the excess positions see nothing).
+ * Two implementations, chosen by shape (pa_prefill_uses_tensor_cores):
+ *  - tensor cores (bf16 pools, head_dim 64 or 128, block_size 8, 16 or 32, and
+ *    128 divisible by the group g = num_heads / num_kv_heads): 128 query rows
+ *    (128 / g new tokens x g heads of one kv head) per tile, S = Q.K^T and
+ *    O += P.V as tcgen05 MMAs with the accumulators in tensor memory, P as a
+ *    bf16 pair hi + lo (about 16 significant bits), partition_size unused.
+ *    K/V inside a tile are read once for all its rows, so every visible K/V
+ *    value must be finite: a non-finite value at position t reaches every row of
+ *    the tile (rows before t included); slots past the last visible position and
+ *    free blocks may still hold anything.
+ *  - otherwise each new token is one query row of the decode kernels, with its
+ *    context cut at its own position; consecutive new tokens of a sequence share
+ *    every whole partition and are served together (up to 8 / group per K/V read).
  */
 PA_API size_t pa_prefill_workspace_bytes(int num_tokens, int num_heads, int head_dim,
                                          int max_context_len, int partition_size);
+/* 1 if pa_prefill serves this shape on the tensor cores, 0 if by decode rows. */
+PA_API int pa_prefill_uses_tensor_cores(pa_dtype dtype, int num_heads, int num_kv_heads, int head_dim,
+                                        int block_size);
 PA_API int pa_prefill(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
                       const int32_t* query_start, int num_seqs, int num_tokens, int num_heads,

@@ -44,16 +44,11 @@
 
 #include "pa_device.cuh"
 #include "pa_host.h"
+#include "pa_tma.h"
+#include "prefill_tc.h"
 
 namespace pa {
 
-constexpr float NEG_INF = -INFINITY;
-constexpr float LOG2E = 1.4426950408889634f;
-// Lazy rescaling: the running max of a head is only raised when a tile's max
-// exceeds it by more than this many powers of two, so most tiles skip the
-// rescale of the accumulators.  Weights stay <= 2^8 -- harmless in fp32 and
-// exact-range in bf16; the final quotient is unchanged.
-constexpr float RESCALE_THRESHOLD = 8.0f;
 
 struct DecodeArgs {
     void* out;
@@ -97,42 +92,12 @@ __device__ __forceinline__ void split_item(int item, int max_parts, int& s, int&
     p = sp - s * max_parts;
 }
 
-__device__ __forceinline__ int clamp_context(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
 
 // ---------------------------------------------------------------------------
 // 1. plan
 // ---------------------------------------------------------------------------
 
 constexpr int PLAN_THREADS = 1024;
-
-__device__ __forceinline__ int warp_inclusive_scan(int v) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(FULL_MASK, v, o);
-        if (lane >= o) v += n;
-    }
-    return v;
-}
-
-// Exclusive prefix sum of v over the CTA; *total receives the sum.
-// `scratch` holds 33 ints.
-__device__ int cta_exclusive_scan(int v, int* total, int* scratch) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const int inc = warp_inclusive_scan(v);
-    __syncthreads();
-    if (lane == 31) scratch[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        const int x = lane < nw ? scratch[lane] : 0;
-        const int xi = warp_inclusive_scan(x);
-        if (lane < nw) scratch[lane] = xi - x;
-        if (lane == 31) scratch[32] = xi;
-    }
-    __syncthreads();
-    *total = scratch[32];
-    return scratch[warp] + inc - v;
-}
 
 // Number of leading whole partitions that sequence s (context c) shares with
 // s + 1 (context c_next): the partitions whose block-table entries name the
@@ -950,41 +915,6 @@ inline int parts_for(int cap, int P) {
     return n < 1 ? 1 : n;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline EncodeTiledFn encode_tiled_fn() {
-    static std::atomic<EncodeTiledFn> fn{nullptr};
-    EncodeTiledFn f = fn.load(std::memory_order_acquire);
-    if (f) return f;
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || ptr == nullptr)
-        return nullptr;
-    f = reinterpret_cast<EncodeTiledFn>(ptr);
-    fn.store(f, std::memory_order_release);
-    return f;
-}
-
-// Tensor map over one bf16 pool viewed as rows of head_dim elements
-// (row = (block * Hkv + kv_head) * B + slot), boxes of 64 columns x rb rows.
-inline bool encode_pool_map(CUtensorMap* m, const void* pool, int num_blocks, int Hkv, int B, int D,
-                            int rb) {
-    EncodeTiledFn enc = encode_tiled_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D),
-                                static_cast<cuuint64_t>(num_blocks) * Hkv * B};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(rb)};
-    const cuuint32_t estr[2] = {1u, 1u};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int RB>
 int launch_attend_bf16(const DecodeArgs& a, cudaStream_t st, long long unit_bound) {
     using Geo = TileGeom<D, RB>;
@@ -1031,18 +961,10 @@ extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int hea
     return ws_layout(num_seqs, num_heads, head_dim, parts_for(max_context_len, partition_size)).total;
 }
 
-// Shared by decode and prefill; `row_seq` (device, may be null) maps each query
-// row to its block-table row.  `prep` (may be null) launches first, after the
-// validation, to produce row_seq / context_lens for prefill.
-template <typename Prep>
-static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
-                       const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
-                       int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
-                       int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
-                       int partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
-                       int32_t* dev_err, pa_stream stream, int phases, const int32_t* row_seq,
-                       Prep prep) {
-    // ---- host-side validation: nothing is launched unless everything is sane
+// Checks of the shapes and scalars shared by decode and prefill.
+static int check_shapes(pa_dtype out_dtype, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, int max_blocks_per_seq, int max_context_len,
+                        float scale, int partition_size, pa_dtype dtype) {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0)
         return PA_ERR_INVALID_ARG;
@@ -1056,14 +978,39 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
         partition_size % block_size != 0)
         return PA_ERR_UNSUPPORTED;
     if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-    if ((phases & ~PA_PHASE_ALL) != 0 || phases == 0) return PA_ERR_INVALID_ARG;
     if (static_cast<long long>(num_blocks) * num_kv_heads * block_size > INT_MAX)
         return PA_ERR_UNSUPPORTED;   // bulk-copy row coordinates are 32-bit
     if (static_cast<long long>(max_blocks_per_seq) * block_size > INT_MAX) return PA_ERR_INVALID_ARG;
-    if (num_seqs == 0) return PA_OK;
+    return PA_OK;
+}
 
+// Largest context the block tables can address, cut at max_context_len when given.
+static long long context_cap(int max_blocks_per_seq, int block_size, int max_context_len) {
     long long cap = static_cast<long long>(max_blocks_per_seq) * block_size;
     if (max_context_len > 0 && max_context_len < cap) cap = max_context_len;
+    return cap;
+}
+
+// Shared by decode and prefill; `row_seq` (device, may be null) maps each query
+// row to its block-table row.  `prep` (may be null) launches first, after the
+// validation, to produce row_seq / context_lens for prefill.
+template <typename Prep>
+static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
+                       const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                       int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                       int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                       int partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                       int32_t* dev_err, pa_stream stream, int phases, const int32_t* row_seq,
+                       Prep prep) {
+    // ---- host-side validation: nothing is launched unless everything is sane
+    const int shape_rc = check_shapes(out_dtype, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                      num_blocks, max_blocks_per_seq, max_context_len, scale, partition_size,
+                                      dtype);
+    if (shape_rc != PA_OK) return shape_rc;
+    if ((phases & ~PA_PHASE_ALL) != 0 || phases == 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+
+    const long long cap = context_cap(max_blocks_per_seq, block_size, max_context_len);
     const int max_parts = parts_for(static_cast<int>(cap), partition_size);
     if (static_cast<long long>(num_seqs) * max_parts > INT_MAX / 16) return PA_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, max_parts);
@@ -1181,7 +1128,15 @@ extern "C" size_t pa_prefill_workspace_bytes(int num_tokens, int num_heads, int 
                                              int max_context_len, int partition_size) {
     const size_t d = pa_decode_workspace_bytes(num_tokens, num_heads, head_dim, max_context_len,
                                                partition_size);
-    return d == 0 ? 0 : prefill_rows_bytes(num_tokens) + d;
+    if (d == 0) return 0;
+    const size_t rows = prefill_rows_bytes(num_tokens) + d;   // the per-token-row path
+    const size_t tc = prefill_tc_workspace_bytes(num_tokens);  // the tensor-core path
+    return rows > tc ? rows : tc;
+}
+
+extern "C" int pa_prefill_uses_tensor_cores(pa_dtype dtype, int num_heads, int num_kv_heads, int head_dim,
+                                            int block_size) {
+    return prefill_tc_eligible(dtype, num_heads, num_kv_heads, head_dim, block_size) ? 1 : 0;
 }
 
 extern "C" int pa_prefill(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,
@@ -1196,6 +1151,21 @@ extern "C" int pa_prefill(void* out, pa_dtype out_dtype, const void* q, const vo
     if (num_seqs == 0 || !context_lens || !query_start || !workspace) return PA_ERR_INVALID_ARG;
     if (!aligned_to(context_lens, 4) || !aligned_to(query_start, 4) || !aligned_to(workspace, 256))
         return PA_ERR_INVALID_ARG;
+    if (prefill_tc_eligible(dtype, num_heads, num_kv_heads, head_dim, block_size)) {
+        const int rc = check_shapes(out_dtype, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                    num_blocks, max_blocks_per_seq, max_context_len, scale, partition_size,
+                                    dtype);
+        if (rc != PA_OK) return rc;
+        if (!out || !q || !k_cache || !v_cache || !block_tables) return PA_ERR_INVALID_ARG;
+        if (!aligned_to(out, 16) || !aligned_to(q, 16) || !aligned_to(k_cache, 16) ||
+            !aligned_to(v_cache, 16) || !aligned_to(block_tables, 4))
+            return PA_ERR_INVALID_ARG;
+        const long long cap = context_cap(max_blocks_per_seq, block_size, max_context_len);
+        return prefill_tc(out, out_dtype, q, k_cache, v_cache, block_tables, context_lens, query_start, num_seqs,
+                          num_tokens, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                          max_blocks_per_seq, static_cast<int>(cap), scale, workspace, workspace_bytes, dev_err,
+                          as_stream(stream));
+    }
     const size_t rows = prefill_rows_bytes(num_tokens);
     if (workspace_bytes < rows) return PA_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);

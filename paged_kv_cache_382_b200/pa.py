@@ -36,6 +36,7 @@ SIGNATURES = {
     "pa_decode_phases": (_i, _DECODE_ARGS + [_i]),
     "pa_copy_blocks": (_i, [_vp, _vp, _i64p, _i, _sz, _i, _i32p, _vp]),
     "pa_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "pa_prefill_uses_tensor_cores": (_i, [_i, _i, _i, _i, _i]),
     "pa_prefill": (_i, [_vp, _i, _vp, _vp, _vp, _i32p, _i32p, _i32p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                         _i, _vp, _sz, _i, _i32p, _vp]),
     "pa_decode_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i32p, _i32p, _i, _i, _i, _i, _i, _i, _i, _i, _f,
@@ -212,6 +213,13 @@ def prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: 
         _stream_handle(stream))
     _check(rc, "pa_prefill")
     return out
+
+
+def prefill_uses_tensor_cores(dtype: torch.dtype, num_heads: int, num_kv_heads: int, head_dim: int,
+                              block_size: int) -> bool:
+    """Whether ``prefill`` serves this shape with the tensor-core (tcgen05) kernel."""
+    return bool(lib.pa_prefill_uses_tensor_cores(dtype_code(dtype), num_heads, num_kv_heads, head_dim,
+                                                 block_size))
 
 
 def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: torch.Tensor,

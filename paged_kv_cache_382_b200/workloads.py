@@ -346,6 +346,25 @@ def prefill_flops(step: DecodeStep) -> int:
     return 4 * step.head_dim * step.num_heads * total
 
 
+def prefill_tc_mma_flops(step: DecodeStep, rows: int = 128, tile: int = 32) -> int:
+    """Tensor-core flops the tcgen05 prefill issues: per tile of 128 query rows x
+    32 tokens, S = Q.K^T (2*128*32*d) and P.V with P as hi + lo (2 x 2*128*32*d),
+    for every tile a query block reaches (masked positions and padding rows
+    included)."""
+    g = step.num_heads // step.num_kv_heads
+    tq = rows // g
+    tiles = 0
+    qs = step.query_start
+    for s in range(step.num_seqs):
+        n = int(qs[s + 1] - qs[s])
+        c = int(step.context_lens[s])
+        for qb in range(-(-n // tq)):
+            pos_max = c - n + min(n, (qb + 1) * tq) - 1
+            if pos_max >= 0:
+                tiles += pos_max // tile + 1
+    return tiles * step.num_kv_heads * 3 * 2 * rows * tile * step.head_dim
+
+
 WORKLOADS = {
     "tiny": tiny,
     "llama7b": llama7b,

@@ -446,26 +446,43 @@ PREFILL_CASES = [
     ([257, 600], [120, 600], 8, 8, 128, 8, 64),
     ([90, 2049], [17, 31], 16, 2, 128, 32, 512),
     ([513, 80], [9, 80], 64, 8, 64, 4, 32),
+    ([200, 77, 1], [200, 20, 1], 12, 4, 128, 16, 64),     # group 3: no tensor-core tile
+    ([333, 64, 129], [100, 64, 129], 32, 2, 64, 8, 128),  # group 16: 8 tokens per tile
 ]
+
+
+def prefill_inputs(case, dtype, poison=False, seed_q=7):
+    ctx, new, Hq, Hkv, d, B, P = case
+    step = to_device(W.independent("prefill", ctx, dtype=dtype, num_heads=Hq, num_kv_heads=Hkv, head_dim=d,
+                                   block_size=B, seed=sum(new), poison=poison, partition_size=P))
+    gen = torch.Generator(device="cuda").manual_seed(seed_q)
+    T = sum(new)
+    q = torch.empty(T, Hq, d, dtype=torch.float32, device="cuda").normal_(generator=gen).to(dtype)
+    qs = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    return step, q, qs
+
+
+def run_prefill(pa, step, q, qs, tables=None, ctx=None, out_dtype=torch.float32, max_context_len=0):
+    T, Hq, d = q.shape
+    out = torch.full((T, Hq, d), float("nan"), dtype=out_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tables = step.block_tables if tables is None else tables
+    ctx = step.context_lens if ctx is None else ctx
+    pa.prefill(out, q, step.k_cache, step.v_cache,
+               torch.from_numpy(np.ascontiguousarray(tables, dtype=np.int32)).cuda(),
+               torch.from_numpy(np.ascontiguousarray(ctx, dtype=np.int32)).cuda(), torch.from_numpy(qs).cuda(),
+               step.scale, partition_size=step.partition_size, max_context_len=max_context_len, dev_err=err)
+    torch.cuda.synchronize()
+    return out, int(err.item())
 
 
 @pytest.mark.parametrize("case", PREFILL_CASES, ids=lambda c: f"h{c[2]}x{c[3]}_d{c[4]}_b{c[5]}_p{c[6]}")
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 def test_prefill_matches_oracle(pa, case, dtype):
     ctx, new, Hq, Hkv, d, B, P = case
-    step = to_device(W.independent("prefill", ctx, dtype=dtype, num_heads=Hq, num_kv_heads=Hkv, head_dim=d,
-                                   block_size=B, seed=sum(new), poison=False, partition_size=P))
-    gen = torch.Generator(device="cuda").manual_seed(7)
-    T = sum(new)
-    q = torch.empty(T, Hq, d, dtype=torch.float32, device="cuda").normal_(generator=gen).to(dtype)
-    qs = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
-    out = torch.empty(T, Hq, d, dtype=torch.float32, device="cuda")
-    err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    pa.prefill(out, q, step.k_cache, step.v_cache, torch.from_numpy(step.block_tables).cuda(),
-               torch.from_numpy(step.context_lens).cuda(), torch.from_numpy(qs).cuda(), step.scale,
-               partition_size=P, dev_err=err)
-    torch.cuda.synchronize()
-    assert int(err.item()) == 0
+    step, q, qs = prefill_inputs(case, dtype)
+    out, err = run_prefill(pa, step, q, qs)
+    assert err == 0
     ref = oracle.prefill_attention(f64(q), f64(step.k_cache), f64(step.v_cache), step.block_tables,
                                    step.context_lens, qs, step.scale)
     assert_close(f64(out), ref, dtype, torch.float32, str(case))
@@ -475,4 +492,113 @@ def test_prefill_matches_oracle(pa, case, dtype):
     pa.decode(dec, q[last].contiguous(), step.k_cache, step.v_cache, torch.from_numpy(step.block_tables).cuda(),
               torch.from_numpy(step.context_lens).cuda(), step.scale, partition_size=P)
     torch.cuda.synchronize()
-    assert torch.equal(out[last], dec)
+    if pa.prefill_uses_tensor_cores(dtype, Hq, Hkv, d, B):
+        # another kernel, another summation order: equal up to both error bounds
+        assert float((out[last] - dec).abs().max()) <= 2 * TOL_BF16
+    else:
+        # the same decode kernels on the same rows: bit for bit
+        assert torch.equal(out[last], dec)
+
+
+def test_prefill_path_choice(pa):
+    bf, f32 = torch.bfloat16, torch.float32
+    assert pa.prefill_uses_tensor_cores(bf, 32, 8, 128, 16)
+    assert pa.prefill_uses_tensor_cores(bf, 32, 32, 64, 8)
+    assert pa.prefill_uses_tensor_cores(bf, 128, 1, 128, 32)     # group 128: one token per tile
+    assert not pa.prefill_uses_tensor_cores(f32, 32, 8, 128, 16)
+    assert not pa.prefill_uses_tensor_cores(bf, 32, 8, 128, 4)
+    assert not pa.prefill_uses_tensor_cores(bf, 12, 4, 128, 16)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["out_f32", "out_bf16"])
+def test_prefill_tensor_core_bf16_output(pa, out_dtype):
+    case = ([300, 1029, 64, 1], [300, 45, 64, 1], 32, 8, 128, 16, 128)
+    step, q, qs = prefill_inputs(case, torch.bfloat16)
+    out, err = run_prefill(pa, step, q, qs, out_dtype=out_dtype)
+    assert err == 0
+    ref = oracle.prefill_attention(f64(q), f64(step.k_cache), f64(step.v_cache), step.block_tables,
+                                   step.context_lens, qs, step.scale)
+    assert_close(f64(out), ref, torch.bfloat16, out_dtype, "prefill out " + str(out_dtype))
+
+
+def test_prefill_reservation_and_free_blocks_are_ignored(pa):
+    """NaN in every free block and reservation slot: the tensor-core prefill gives
+    the same output as without them, bit for bit, and a finite one."""
+    case = ([7, 40, 100, 333], [7, 3, 33, 100], 16, 4, 128, 16, 64)
+    assert pa.prefill_uses_tensor_cores(torch.bfloat16, 16, 4, 128, 16)
+    clean, q, qs = prefill_inputs(case, torch.bfloat16, poison=False)
+    dirty, _, _ = prefill_inputs(case, torch.bfloat16, poison=True)
+    for st in (clean, dirty):   # the step's own token of each sequence is written first
+        pa.reshape_and_cache(st.new_key, st.new_value, st.k_cache, st.v_cache,
+                             torch.from_numpy(st.slot_mapping).cuda())
+    a, ea = run_prefill(pa, clean, q, qs)
+    b, eb = run_prefill(pa, dirty, q, qs)
+    assert ea == 0 and eb == 0
+    assert torch.isfinite(b).all()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_prefill_more_new_tokens_than_context(pa, dtype):
+    """n_s > context_len is flagged; positions below zero see nothing (zeros), the
+    others are the causal result over what exists."""
+    case = ([40, 50], [10, 20], 8, 2, 64, 16, 32)
+    step, q, qs = prefill_inputs(case, dtype)
+    ctx = np.array([5, 50], dtype=np.int32)       # sequence 0: 10 new tokens but 5 in the pool
+    out, err = run_prefill(pa, step, q, qs, ctx=ctx)
+    assert err & pa.DEVERR_CONTEXT
+    got = f64(out)
+    assert np.all(got[:5] == 0.0)                 # positions -5 .. -1
+    ref = oracle.prefill_attention(f64(q[5:]), f64(step.k_cache), f64(step.v_cache), step.block_tables,
+                                   ctx, np.array([0, 5, 25], dtype=np.int32), step.scale)
+    assert_close(got[5:], ref, dtype, torch.float32, "excess new tokens")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_prefill_bad_block_id_is_flagged(pa, dtype):
+    case = ([64, 64], [16, 16], 8, 2, 64, 16, 32)
+    step, q, qs = prefill_inputs(case, dtype)
+    tables = step.block_tables.copy()
+    tables[1, 1] = step.num_blocks + 5            # tokens 16..31 of sequence 1 live nowhere
+    out, err = run_prefill(pa, step, q, qs, tables=tables)
+    assert err & pa.DEVERR_BLOCK_ID
+    assert torch.isfinite(out).all()
+    ref = oracle.prefill_attention(f64(q[:16]), f64(step.k_cache), f64(step.v_cache), step.block_tables[:1],
+                                   step.context_lens[:1], qs[:2], step.scale)
+    assert_close(f64(out[:16]), ref, dtype, torch.float32, "sequence with valid blocks")
+
+
+def test_prefill_chunk_full_size_sampled(pa):
+    """The chunked-prefill workload timed by the benchmark (16 sequences x (1024
+    cached + 256 new tokens), 32 q / 8 kv heads, d 128, block 16), in the same
+    launch configuration; sampled rows against the oracle one by one."""
+    step = to_device(W.prefill_chunk())
+    T = step.q.shape[0]
+    out = torch.empty(T, step.num_heads, step.head_dim, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qs = step.query_start
+    kc, vc = step.k_cache.clone(), step.v_cache.clone()
+    pa.reshape_and_cache(step.new_key, step.new_value, kc, vc, torch.from_numpy(step.slot_mapping).cuda(),
+                         dev_err=err)
+    pa.prefill(out, step.q, kc, vc, torch.from_numpy(step.block_tables).cuda(),
+               torch.from_numpy(step.context_lens).cuda(), torch.from_numpy(qs).cuda(), step.scale,
+               partition_size=step.partition_size, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rng = np.random.default_rng(3)
+    g = step.num_heads // step.num_kv_heads
+    for s in rng.choice(step.num_seqs, size=4, replace=False):
+        c = int(step.context_lens[s])
+        n = int(qs[s + 1] - qs[s])
+        blocks = step.block_tables[s][: -(-c // step.block_size)]
+        kp = SparsePool.fetch(kc, blocks)
+        vp = SparsePool.fetch(vc, blocks)
+        for i in sorted(set(rng.integers(0, n, size=5).tolist()) | {0, n - 1}):
+            pos = c - n + i
+            row = int(qs[s]) + i
+            for h in rng.choice(step.num_heads, size=4, replace=False):
+                kvh = int(h) // g
+                k_rows = oracle.gather_kv(kp, step.block_tables[s], pos + 1, kvh)
+                v_rows = oracle.gather_kv(vp, step.block_tables[s], pos + 1, kvh)
+                ref = oracle.decode_attention_one(f64(step.q[row, h]), k_rows, v_rows, step.scale)
+                assert_close(f64(out[row, h]), ref, torch.bfloat16, torch.bfloat16, f"seq {s} token {i} head {h}")
