@@ -80,7 +80,13 @@ CONFIGS["host_block_manager"] = dict(
     desc="host block manager (pa_bm_*, C++): 256 requests with a 512-token shared system prompt + "
          "64 user tokens, then 256 decode steps of one token each, block_size 16")
 DEFAULT_CONFIG = "llama7b"
-ATTEND_SOURCES = ["paged_kv_cache_382_b200/csrc/decode.cu", "paged_kv_cache_382_b200/csrc/pa_device.cuh"]
+# sources that make up each profiled kernel: a committed ncu summary counts only
+# while their hash is the one it records
+KERNEL_SOURCES = {
+    "attend": ["paged_kv_cache_382_b200/csrc/decode.cu", "paged_kv_cache_382_b200/csrc/pa_device.cuh"],
+    "prefill_tc": ["paged_kv_cache_382_b200/csrc/prefill_tc.cu", "paged_kv_cache_382_b200/csrc/pa_umma.cuh",
+                   "paged_kv_cache_382_b200/csrc/pa_device.cuh"],
+}
 
 
 def parse_args(argv=None):
@@ -116,18 +122,19 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def attend_source_hash() -> str:
+def kernel_source_hash(kernel: str = "attend") -> str:
     h = hashlib.sha256()
-    for rel in ATTEND_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def profiled_traffic(config: str):
-    """dram bytes per attend launch from the committed ncu summary of this workload,
-    or None if there is none or the kernel source changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"attend_{config}.ncu.md")
+def profiled_traffic(config: str, kernel: str = "attend"):
+    """dram bytes per launch of the kernel from the committed ncu summary of this
+    workload (profiles/<kernel>_<config>.ncu.md), or None if there is none or the
+    kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{config}.ncu.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -137,7 +144,7 @@ def profiled_traffic(config: str):
                 k, v = line.strip()[2:].split(":", 1)
                 fields[k.strip()] = v.strip().strip("`")
     try:
-        if fields.get("kernel_source_sha256") != attend_source_hash():
+        if fields.get("kernel_source_sha256") != kernel_source_hash(kernel):
             return None
         return int(float(fields["dram_bytes_per_launch"]))
     except (KeyError, ValueError):
@@ -577,7 +584,8 @@ def prefill_line(args, step, world, K, max_ms, prefill_ms, alg_bytes, clock_info
                                 else "pa_prefill (decode rows: rows, plan, attend, reduce)"),
                      "bound": "tensor",
                      "achieved": round(tflops_call, 2), "peak": peak, "peak_kind": kind, "unit": "TFLOP/s",
-                     "frac": round(tflops_call / peak, 4), "traffic": None,
+                     "frac": round(tflops_call / peak, 4),
+                     "traffic": (profiled_traffic(args.config, "prefill_tc") if ds.tensor_core_prefill else None),
                      "prefill_ms": round(prefill_ms, 5),
                      "mma_flops_issued": (W.prefill_tc_mma_flops(step) if ds.tensor_core_prefill else None)},
         "clocks": clock_info, "e2e": None, "cpu_baseline": None,

@@ -67,6 +67,10 @@ inline int prepare_kernel(KernelSlot& slot, const void* func, int threads, int s
 #endif
         return -1;
     }
+#ifdef PA_DEBUG_ERRORS
+    fprintf(stderr, "libpa: kernel set-up: %d CTAs/SM of %d threads at %d B shared memory\n", c, threads,
+            smem_bytes);
+#endif
     slot.ctas_per_sm[dev].store(c, std::memory_order_relaxed);
     slot.smem[dev].store(smem_bytes, std::memory_order_release);
     return c;
