@@ -14,13 +14,15 @@
 //           major: row r is new token r / g of the block, head r % g of the
 //           group.  Within a sequence the later blocks, which see more
 //           context, come first.
-//   attend: persistent CTAs take (item, kv head) units from an atomic ticket.
-//           A unit streams the K/V it can see in tiles of 32 tokens (one
-//           tensor-map bulk copy per block and 64-column half, 128-byte
-//           swizzle) through a 3-stage ring.  Warp 5 issues the copies as
-//           soon as a stage is free; one thread of warp 4 issues the MMAs,
-//           each as soon as its inputs are ready (it polls, so a copy still in
-//           flight never holds back a P.V whose weights are written):
+//   attend: persistent CTAs (two per SM, each with half of the tensor
+//           memory) take (item, kv head) units from an atomic ticket.  A unit
+//           streams the K/V it can see in tiles of 32 tokens (one tensor-map
+//           bulk copy per block and 64-column half, 128-byte swizzle) through
+//           a 4-stage ring.  Warp 5 issues the copies as soon as a stage is
+//           free, reading the block table 32 entries at a time across its
+//           lanes; one thread of warp 4 issues the MMAs, each as soon as its
+//           inputs are ready (it polls, so a copy still in flight never holds
+//           back a P.V whose weights are written):
 //             S = Q . K^T   (M = 128 rows, N = 32 tokens, K = d) into a ring of
 //                            four TMEM buffers;
 //             O += P . V    (M = 128, N = d, K = 32 tokens, P as bf16 hi + lo
@@ -331,17 +333,31 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             }
         } else if (compute_warp) {
             // Q tile: row r = new token tok0 + r / G, head kvh * G + r % G; rows past
-            // the unit's tokens are zero
-            for (int idx = tid; idx < TC_ROWS * (D / 8); idx += TC_COMPUTE_WARPS * 32) {
-                const int row = idx / (D / 8), ch = idx - (idx / (D / 8)) * (D / 8);
-                const int t = row / G;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (t < ntok) {
-                    const size_t qrow = static_cast<size_t>(first + tok0 + t) * a.num_heads + kvh * G + row % G;
-                    v = __ldg(reinterpret_cast<const uint4*>(a.q + qrow * D) + ch);
+            // the unit's tokens are zero.  All loads are issued before the first
+            // store (one round trip), in two batches to bound the registers.
+            constexpr int QLOADS = TC_ROWS * (D / 8) / (TC_COMPUTE_WARPS * 32);
+            constexpr int QBATCH = QLOADS < 8 ? QLOADS : 8;
+#pragma unroll
+            for (int k0 = 0; k0 < QLOADS; k0 += QBATCH) {
+                uint4 qv[QBATCH];
+#pragma unroll
+                for (int k = 0; k < QBATCH; ++k) {
+                    const int idx = tid + (k0 + k) * (TC_COMPUTE_WARPS * 32);
+                    const int row = idx / (D / 8), ch = idx % (D / 8);
+                    const int t = row / G;
+                    qv[k] = make_uint4(0u, 0u, 0u, 0u);
+                    if (t < ntok) {
+                        const size_t qrow = static_cast<size_t>(first + tok0 + t) * a.num_heads + kvh * G + row % G;
+                        qv[k] = __ldg(reinterpret_cast<const uint4*>(a.q + qrow * D) + ch);
+                    }
                 }
-                *reinterpret_cast<uint4*>(smem + Geo::OFF_Q + (ch / 8) * Geo::Q_HALF + row * 128 +
-                                          (((ch % 8) ^ (row & 7)) << 4)) = v;
+#pragma unroll
+                for (int k = 0; k < QBATCH; ++k) {
+                    const int idx = tid + (k0 + k) * (TC_COMPUTE_WARPS * 32);
+                    const int row = idx / (D / 8), ch = idx % (D / 8);
+                    *reinterpret_cast<uint4*>(smem + Geo::OFF_Q + (ch / 8) * Geo::Q_HALF + row * 128 +
+                                              (((ch % 8) ^ (row & 7)) << 4)) = qv[k];
+                }
             }
             fence_proxy_async_smem();   // Q is read by the MMAs (async proxy)
             named_barrier_sync(TC_Q_BARRIER, TC_Q_BARRIER_THREADS);
