@@ -322,6 +322,17 @@ PA_API int pa_bm_num_free(const pa_block_manager* manager);
 /* -1 for a bad block id. */
 PA_API int pa_bm_ref_count(const pa_block_manager* manager, int block);
 
+/*
+ * pa_selftest_bounded_wait -- checks, on the device, the bounded wait that every
+ * wait of libpa's kernels for an asynchronous copy or tensor-core operation uses
+ * (see "Errors" above): one warp waits on a shared-memory barrier that nothing
+ * ever arrives at.  After limit_ns (0 < limit_ns <= 10^9) it must give up, OR
+ * PA_DEVERR_TIMEOUT into *dev_err (device, required) and return, leaving the
+ * context usable.  Asynchronous on `stream`.  The pages have no counterpart; it
+ * exists so the timeout path can be tested without a fault.
+ */
+PA_API int pa_selftest_bounded_wait(int32_t* dev_err, uint64_t limit_ns, pa_stream stream);
+
 /* Human-readable name of a pa_status value (static storage). */
 PA_API const char* pa_status_string(int status);
 

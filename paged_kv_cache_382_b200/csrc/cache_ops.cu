@@ -70,7 +70,29 @@ copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
     }
 }
 
+// Self-test of the bounded wait every asynchronous-copy wait of libpa goes
+// through: a barrier that nothing ever arrives at must be given up on after
+// `limit_ns`, with PA_DEVERR_TIMEOUT raised, and the kernel must return.
+__global__ void __launch_bounds__(32) selftest_wait_kernel(uint64_t limit_ns, int32_t* dev_err) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (!mbar_wait_bounded(smem_u32(&bar), 0, limit_ns) && threadIdx.x == 0)
+        flag_error(dev_err, PA_DEVERR_TIMEOUT);
+}
+
 }  // namespace pa
+
+extern "C" int pa_selftest_bounded_wait(int32_t* dev_err, uint64_t limit_ns, pa_stream stream) {
+    using namespace pa;
+    if (!dev_err || !aligned_to(dev_err, 4) || limit_ns == 0 || limit_ns > 1000000000ull)
+        return PA_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns, dev_err);
+    return launch_status(cudaGetLastError());
+}
 
 extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_cache,
                                     void* v_cache, const int64_t* slot_mapping, int num_tokens,

@@ -52,6 +52,7 @@ SIGNATURES = {
                                ctypes.POINTER(ctypes.c_int64)]),
     "pa_bm_num_free": (_i, [_vp]),
     "pa_bm_ref_count": (_i, [_vp, _i]),
+    "pa_selftest_bounded_wait": (_i, [_i32p, ctypes.c_uint64, _vp]),
     "pa_status_string": (ctypes.c_char_p, [_i]),
     "pa_version": (_i, []),
 }
@@ -220,6 +221,14 @@ def prefill_uses_tensor_cores(dtype: torch.dtype, num_heads: int, num_kv_heads: 
     """Whether ``prefill`` serves this shape with the tensor-core (tcgen05) kernel."""
     return bool(lib.pa_prefill_uses_tensor_cores(dtype_code(dtype), num_heads, num_kv_heads, head_dim,
                                                  block_size))
+
+
+def selftest_bounded_wait(dev_err: torch.Tensor, limit_ns: int = 1_000_000,
+                          stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Launch the device self-test of the bounded wait: it must OR
+    DEVERR_TIMEOUT into dev_err after limit_ns and return."""
+    rc = lib.pa_selftest_bounded_wait(_dev(dev_err, "dev_err", torch.int32), int(limit_ns), _stream_handle(stream))
+    _check(rc, "pa_selftest_bounded_wait")
 
 
 def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: torch.Tensor,

@@ -374,6 +374,21 @@ def test_packed_shared_prefix_units_are_bit_identical(pa, heads):
     assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, f"packed {heads}")
 
 
+def test_bounded_wait_gives_up_and_the_context_survives(pa):
+    """The bounded wait all asynchronous-copy waits use: a barrier nothing arrives
+    at is given up on after the limit, PA_DEVERR_TIMEOUT is raised, the kernel
+    returns, and the context keeps working (a decode step afterwards is exact)."""
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.selftest_bounded_wait(err, limit_ns=2_000_000)
+    torch.cuda.synchronize()
+    assert int(err.item()) == pa.DEVERR_TIMEOUT
+    step = to_device(W.tiny(block_size=16, poison=True))
+    out, *_, e, _ = run_gpu(pa, step)
+    assert e == 0
+    err_max = float(np.abs(f64(out) - full_oracle(step)).max())
+    assert err_max < TOL_F32
+
+
 def test_single_token_context_returns_the_value_row(pa):
     step = to_device(W.independent("one", [1, 1, 1], dtype=torch.bfloat16, num_heads=8, num_kv_heads=2,
                                    head_dim=128, block_size=8, seed=2))

@@ -55,6 +55,15 @@ def test_status_strings_and_version(pa):
     assert pa.lib.pa_version() >= 100
 
 
+def test_selftest_host_validation(pa):
+    """Bad arguments of the bounded-wait self-test are refused before any launch."""
+    f = pa.lib.pa_selftest_bounded_wait
+    assert f(None, 1000, None) == pa.PA_ERR_INVALID_ARG              # no error word
+    assert f(256, 0, None) == pa.PA_ERR_INVALID_ARG                  # no limit
+    assert f(256, 2_000_000_000, None) == pa.PA_ERR_INVALID_ARG      # limit above 1 s
+    assert f(258, 1000, None) == pa.PA_ERR_INVALID_ARG               # misaligned error word
+
+
 def test_workspace_bytes(pa):
     ws = pa.lib.pa_decode_workspace_bytes
     # one partition: header + work list only
