@@ -463,6 +463,8 @@ PREFILL_CASES = [
     ([513, 80], [9, 80], 64, 8, 64, 4, 32),
     ([200, 77, 1], [200, 20, 1], 12, 4, 128, 16, 64),     # group 3: no tensor-core tile
     ([333, 64, 129], [100, 64, 129], 32, 2, 64, 8, 128),  # group 16: 8 tokens per tile
+    ([77, 40, 300], [13, 0, 37], 64, 2, 64, 16, 64),      # group 32: 4 tokens per tile; an empty sequence
+    ([50, 33], [9, 33], 128, 1, 64, 32, 32),              # group 128: one token per tile
 ]
 
 
@@ -502,10 +504,12 @@ def test_prefill_matches_oracle(pa, case, dtype):
                                    step.context_lens, qs, step.scale)
     assert_close(f64(out), ref, dtype, torch.float32, str(case))
     # the last new token of each sequence sees its whole context: it is the decode result
-    last = torch.from_numpy(qs[1:] - 1).long().cuda()
-    dec = torch.empty(len(ctx), Hq, d, dtype=torch.float32, device="cuda")
-    pa.decode(dec, q[last].contiguous(), step.k_cache, step.v_cache, torch.from_numpy(step.block_tables).cuda(),
-              torch.from_numpy(step.context_lens).cuda(), step.scale, partition_size=P)
+    nz = np.array([i for i in range(len(ctx)) if new[i] > 0])
+    last = torch.from_numpy(qs[1:][nz] - 1).long().cuda()
+    dec = torch.empty(len(nz), Hq, d, dtype=torch.float32, device="cuda")
+    pa.decode(dec, q[last].contiguous(), step.k_cache, step.v_cache,
+              torch.from_numpy(np.ascontiguousarray(step.block_tables[nz])).cuda(),
+              torch.from_numpy(np.ascontiguousarray(step.context_lens[nz])).cuda(), step.scale, partition_size=P)
     torch.cuda.synchronize()
     if pa.prefill_uses_tensor_cores(dtype, Hq, Hkv, d, B):
         # another kernel, another summation order: equal up to both error bounds
@@ -513,6 +517,23 @@ def test_prefill_matches_oracle(pa, case, dtype):
     else:
         # the same decode kernels on the same rows: bit for bit
         assert torch.equal(out[last], dec)
+
+
+def test_prefill_many_sequences_plan_chunks(pa):
+    """1500 sequences (the plan kernel walks them 1024 at a time), 1-3 new tokens
+    each over short contexts, on the tensor-core path."""
+    rng = np.random.default_rng(8)
+    S = 1500
+    new = rng.integers(1, 4, size=S)
+    ctx = new + rng.integers(0, 40, size=S)
+    case = (ctx.tolist(), new.tolist(), 8, 2, 64, 16, 32)
+    assert pa.prefill_uses_tensor_cores(torch.bfloat16, 8, 2, 64, 16)
+    step, q, qs = prefill_inputs(case, torch.bfloat16)
+    out, err = run_prefill(pa, step, q, qs)
+    assert err == 0
+    ref = oracle.prefill_attention(f64(q), f64(step.k_cache), f64(step.v_cache), step.block_tables,
+                                   step.context_lens, qs, step.scale)
+    assert_close(f64(out), ref, torch.bfloat16, torch.float32, "1500 sequences")
 
 
 def test_prefill_path_choice(pa):
