@@ -374,6 +374,58 @@ def test_packed_shared_prefix_units_are_bit_identical(pa, heads):
     assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, f"packed {heads}")
 
 
+def random_fork_step(seed, Hq, Hkv, d, B, P, adjacent=True):
+    """A batch whose block tables come from a random serving history through the
+    block manager: prompts, forks at random points (a child shares every block
+    of its parent up to the fork, then diverges, mid-block included) and ragged
+    appends.  Children sit next to their parents (packing applies) unless
+    `adjacent` is false.  The pool holds random values in every block."""
+    from paged_kv_cache_382_b200.blocks import BlockManager, BlockPool, block_table_array
+
+    rng = np.random.default_rng(seed)
+    NB = 600
+    mgr = BlockManager(BlockPool(NB, rng.permutation(NB)), B)
+    seqs = []
+    for _ in range(3):                       # prompts
+        sq = mgr.new_sequence()
+        mgr.append_tokens(sq, int(rng.integers(1, 200)))
+        seqs.append(sq)
+    for _ in range(12):                      # forks with their own continuations
+        i = int(rng.integers(0, len(seqs)))
+        child = mgr.fork(seqs[i])
+        mgr.append_tokens(child, int(rng.integers(0, 90)))
+        seqs.insert(i + 1 if adjacent else len(seqs), child)
+    for sq in seqs:                          # every sequence gets this step's token
+        mgr.append_tokens(sq, 1)
+    gen = torch.Generator(device="cuda").manual_seed(seed)
+    normal = lambda *shape: torch.empty(*shape, dtype=torch.float32, device="cuda").normal_(generator=gen).to(
+        torch.bfloat16)  # noqa: E731
+    S = len(seqs)
+    return W.DecodeStep(
+        name=f"random_fork_{seed}", dtype=torch.bfloat16, num_heads=Hq, num_kv_heads=Hkv, head_dim=d, block_size=B,
+        num_blocks=NB, context_lens=np.array([sq.num_tokens for sq in seqs], dtype=np.int32),
+        block_tables=block_table_array(seqs), scale=float(np.float32(1.0 / math.sqrt(d))), partition_size=P,
+        q=normal(S, Hq, d), k_cache=normal(NB, Hkv, B, d), v_cache=normal(NB, Hkv, B, d),
+        new_key=normal(S, Hkv, d), new_value=normal(S, Hkv, d),
+        slot_mapping=np.full(S, -1, dtype=np.int64), copy_pairs=np.zeros((0, 2), dtype=np.int64))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+@pytest.mark.parametrize("heads", [(16, 4), (8, 4), (8, 8)], ids=["g4", "g2", "g1"])
+def test_random_fork_histories(pa, seed, heads):
+    """Random sharing patterns (shared spans ending anywhere, packed runs of every
+    length, siblings adjacent or not): equal to the oracle, and bit for bit to the
+    same batch without shared block ids."""
+    Hq, Hkv = heads
+    for adjacent in (True, False):
+        step = random_fork_step(seed, Hq, Hkv, 128, 16, 32, adjacent)
+        out, *_, err, _ = run_gpu(pa, step)
+        assert err == 0
+        assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, f"seed {seed} {heads} {adjacent}")
+        out2, *_ = run_gpu(pa, unshared_copy(step))
+        assert torch.equal(out, out2)
+
+
 def test_bounded_wait_gives_up_and_the_context_survives(pa):
     """The bounded wait all asynchronous-copy waits use: a barrier nothing arrives
     at is given up on after the limit, PA_DEVERR_TIMEOUT is raised, the kernel
