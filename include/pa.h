@@ -316,6 +316,20 @@ PA_API int pa_bm_append(pa_block_manager* manager, int64_t seq_id, const int32_t
                         int* num_copies, int* num_cached_tokens);
 /* The sequence's block table (out may be NULL to query *num_blocks); PA_ERR_WORKSPACE if
  * it has more than max_blocks entries.  *num_tokens (nullable) gets its length. */
+/*
+ * pa_bm_append_batch -- pa_bm_append for many sequences in one call (one decode
+ * step of a batch: num_seqs sequences, counts[k] tokens for seq_ids[k]).
+ * token_ids and slots are the concatenation of the per-sequence arrays, in
+ * order; copies[2 * max_copies] collects every sequence's copy-on-write pairs
+ * (run them all before the step's writes), *num_copies their number,
+ * *num_cached_tokens (nullable) the total served from the cache.  All ids and
+ * counts are checked before anything changes (PA_ERR_INVALID_ARG).  On
+ * PA_ERR_WORKSPACE the sequences before the failing one are appended, the
+ * failing one as pa_bm_append leaves it.
+ */
+PA_API int pa_bm_append_batch(pa_block_manager* manager, int num_seqs, const int64_t* seq_ids,
+                              const int32_t* counts, const int32_t* token_ids, int64_t* slots,
+                              int64_t* copies, int max_copies, int* num_copies, int* num_cached_tokens);
 PA_API int pa_bm_block_table(const pa_block_manager* manager, int64_t seq_id, int32_t* out,
                              int max_blocks, int* num_blocks, int64_t* num_tokens);
 PA_API int pa_bm_num_free(const pa_block_manager* manager);

@@ -163,18 +163,14 @@ extern "C" int pa_bm_free(pa_block_manager* m, int64_t seq_id) {
     return PA_OK;
 }
 
-extern "C" int pa_bm_append(pa_block_manager* m, int64_t seq_id, const int32_t* token_ids, int num_tokens,
-                            int64_t* slots, int64_t* copies, int max_copies, int* num_copies,
-                            int* num_cached_tokens) {
-    if (!m || num_tokens < 0 || (num_tokens > 0 && !slots) || max_copies < 0 || !num_copies)
-        return PA_ERR_INVALID_ARG;
-    if (m->prefix_cache && num_tokens > 0 && !token_ids) return PA_ERR_INVALID_ARG;
-    auto it = m->seqs.find(seq_id);
-    if (it == m->seqs.end()) return PA_ERR_INVALID_ARG;
-    Sequence& sq = it->second;
+namespace {
+
+// Appends n tokens to sq; slots[n] gets their slots, copies (room for
+// max_copies pairs) the copy-on-write pairs, counted into *num_copies;
+// *cached (nullable) counts the tokens found in the prefix cache.
+int append_tokens(pa_block_manager* m, Sequence& sq, const int32_t* token_ids, int num_tokens, int64_t* slots,
+                  int64_t* copies, int max_copies, int* num_copies, int* cached) {
     const int B = m->block_size;
-    *num_copies = 0;
-    if (num_cached_tokens) *num_cached_tokens = 0;
     int i = 0;
     while (i < num_tokens) {
         const int64_t pos = sq.num_tokens;
@@ -197,7 +193,7 @@ extern "C" int pa_bm_append(pa_block_manager* m, int64_t seq_id, const int32_t* 
                         for (int k = 0; k < B; ++k) slots[i + k] = -1;   // already in the pool
                         sq.num_tokens += B;
                         i += B;
-                        if (num_cached_tokens) *num_cached_tokens += B;
+                        if (cached) *cached += B;
                         continue;
                     }
                 }
@@ -208,9 +204,9 @@ extern "C" int pa_bm_append(pa_block_manager* m, int64_t seq_id, const int32_t* 
         } else {
             int32_t b = sq.table[logical];
             if (m->ref_cnt[b] > 1) {   // copy on write
+                if (*num_copies >= max_copies) return PA_ERR_WORKSPACE;
                 const int32_t fresh = m->allocate();
                 if (fresh < 0) return PA_ERR_WORKSPACE;
-                if (*num_copies >= max_copies) return PA_ERR_WORKSPACE;
                 if (copies) {
                     copies[2 * *num_copies] = b;
                     copies[2 * *num_copies + 1] = fresh;
@@ -239,6 +235,46 @@ extern "C" int pa_bm_append(pa_block_manager* m, int64_t seq_id, const int32_t* 
         }
         ++sq.num_tokens;
         ++i;
+    }
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_bm_append(pa_block_manager* m, int64_t seq_id, const int32_t* token_ids, int num_tokens,
+                            int64_t* slots, int64_t* copies, int max_copies, int* num_copies,
+                            int* num_cached_tokens) {
+    if (!m || num_tokens < 0 || (num_tokens > 0 && !slots) || max_copies < 0 || !num_copies)
+        return PA_ERR_INVALID_ARG;
+    if (m->prefix_cache && num_tokens > 0 && !token_ids) return PA_ERR_INVALID_ARG;
+    auto it = m->seqs.find(seq_id);
+    if (it == m->seqs.end()) return PA_ERR_INVALID_ARG;
+    *num_copies = 0;
+    if (num_cached_tokens) *num_cached_tokens = 0;
+    return append_tokens(m, it->second, token_ids, num_tokens, slots, copies, max_copies, num_copies,
+                         num_cached_tokens);
+}
+
+extern "C" int pa_bm_append_batch(pa_block_manager* m, int num_seqs, const int64_t* seq_ids,
+                                  const int32_t* counts, const int32_t* token_ids, int64_t* slots,
+                                  int64_t* copies, int max_copies, int* num_copies, int* num_cached_tokens) {
+    if (!m || num_seqs < 0 || (num_seqs > 0 && (!seq_ids || !counts)) || max_copies < 0 || !num_copies)
+        return PA_ERR_INVALID_ARG;
+    int64_t total = 0;
+    for (int k = 0; k < num_seqs; ++k) {   // everything checked before anything changes
+        if (counts[k] < 0 || !m->seqs.count(seq_ids[k])) return PA_ERR_INVALID_ARG;
+        total += counts[k];
+    }
+    if (total > 0 && !slots) return PA_ERR_INVALID_ARG;
+    if (m->prefix_cache && total > 0 && !token_ids) return PA_ERR_INVALID_ARG;
+    *num_copies = 0;
+    if (num_cached_tokens) *num_cached_tokens = 0;
+    int64_t at = 0;
+    for (int k = 0; k < num_seqs; ++k) {
+        const int rc = append_tokens(m, m->seqs.find(seq_ids[k])->second, token_ids ? token_ids + at : nullptr,
+                                     counts[k], slots + at, copies, max_copies, num_copies, num_cached_tokens);
+        if (rc != PA_OK) return rc;
+        at += counts[k];
     }
     return PA_OK;
 }

@@ -48,6 +48,8 @@ SIGNATURES = {
     "pa_bm_free": (_i, [_vp, ctypes.c_int64]),
     "pa_bm_append": (_i, [_vp, ctypes.c_int64, _vp, _i, _vp, _vp, _i, ctypes.POINTER(ctypes.c_int),
                           ctypes.POINTER(ctypes.c_int)]),
+    "pa_bm_append_batch": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, ctypes.POINTER(ctypes.c_int),
+                                ctypes.POINTER(ctypes.c_int)]),
     "pa_bm_block_table": (_i, [_vp, ctypes.c_int64, _vp, _i, ctypes.POINTER(ctypes.c_int),
                                ctypes.POINTER(ctypes.c_int64)]),
     "pa_bm_num_free": (_i, [_vp]),
@@ -323,6 +325,31 @@ class NativeBlockManager:
         _check(rc, "pa_bm_append")
         pairs = [(int(copies[2 * i]), int(copies[2 * i + 1])) for i in range(ncopies.value)]
         return slots[:n], pairs, ncached.value
+
+    def append_batch(self, seq_ids, tokens, max_copies=None):
+        """One call for a batch: tokens[k] (a count, or token ids when prefix
+        caching) appended to seq_ids[k].  Returns (slots of all new tokens in
+        order, [(src, dst) copies], tokens served from the cache)."""
+        np = self._np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        if all(isinstance(t, (int, np.integer)) for t in tokens):
+            counts = np.ascontiguousarray(tokens, dtype=np.int32)
+            toks = None
+        else:
+            counts = np.array([len(t) for t in tokens], dtype=np.int32)
+            toks = np.ascontiguousarray(np.concatenate([np.asarray(t, dtype=np.int32) for t in tokens])
+                                        if len(tokens) else np.zeros(0, dtype=np.int32), dtype=np.int32)
+        total = int(counts.sum())
+        slots = np.empty(max(total, 1), dtype=np.int64)
+        cap = max(total, 1) if max_copies is None else int(max_copies)
+        copies = np.empty(2 * max(cap, 1), dtype=np.int64)
+        ncopies, ncached = ctypes.c_int(0), ctypes.c_int(0)
+        rc = lib.pa_bm_append_batch(self._h, len(ids), ids.ctypes.data, counts.ctypes.data,
+                                    None if toks is None else toks.ctypes.data, slots.ctypes.data,
+                                    copies.ctypes.data, cap, ctypes.byref(ncopies), ctypes.byref(ncached))
+        _check(rc, "pa_bm_append_batch")
+        pairs = [(int(copies[2 * i]), int(copies[2 * i + 1])) for i in range(ncopies.value)]
+        return slots[:total], pairs, ncached.value
 
     def block_table(self, seq_id: int):
         np = self._np

@@ -151,3 +151,55 @@ def test_errors(pa):
     assert pa.lib.pa_bm_create(0, 4, None, 0) is None
     bad = np.array([0, 0], dtype=np.int32)
     assert pa.lib.pa_bm_create(2, 4, bad.ctypes.data, 0) is None
+
+
+@pytest.mark.parametrize("prefix_cache", [False, True], ids=["plain", "prefix_cache"])
+def test_append_batch_equals_one_call_per_sequence(pa, prefix_cache):
+    """pa_bm_append_batch gives the same slots, copy-on-write pairs, cached counts
+    and resulting tables as one pa_bm_append per sequence, in order."""
+    rng = np.random.default_rng(11)
+    NB, B = 400, 16
+    a = pa.NativeBlockManager(NB, B, prefix_cache=prefix_cache)
+    b = pa.NativeBlockManager(NB, B, prefix_cache=prefix_cache)
+    system = rng.integers(1, 1000, size=40).tolist()
+    seqs = []
+    for sid in range(6):                                   # prompts, some with a shared system prompt
+        toks = (system if sid % 2 == 0 else []) + rng.integers(1, 1000, size=int(rng.integers(1, 30))).tolist()
+        for m in (a, b):
+            m.add(sid)
+        ra, rb = a.append(sid, toks if prefix_cache else len(toks)), b.append_batch([sid], [toks if prefix_cache
+                                                                                       else len(toks)])
+        assert list(ra[0]) == list(rb[0]) and ra[1] == rb[1] and ra[2] == rb[2]
+        seqs.append(sid)
+    for child, parent in [(6, 0), (7, 0), (8, 3)]:       # parallel samples
+        a.fork(parent, child)
+        b.fork(parent, child)
+        seqs.append(child)
+    for step in range(12):                                 # decode steps: 1-3 tokens per sequence
+        batch = [rng.integers(1, 1000, size=int(rng.integers(1, 4))).tolist() for _ in seqs]
+        want_slots, want_copies, want_cached = [], [], 0
+        for sid, toks in zip(seqs, batch):
+            s, c, k = a.append(sid, toks if prefix_cache else len(toks))
+            want_slots += list(s)
+            want_copies += c
+            want_cached += k
+        got_slots, got_copies, got_cached = b.append_batch(seqs, batch if prefix_cache else [len(t) for t in batch])
+        assert list(got_slots) == want_slots and got_copies == want_copies and got_cached == want_cached
+    for sid in seqs:
+        assert a.block_table(sid) == b.block_table(sid)
+    assert a.num_free == b.num_free
+
+
+def test_append_batch_validation(pa):
+    m = pa.NativeBlockManager(8, 4)
+    m.add(0)
+    with pytest.raises(Exception):
+        m.append_batch([0, 5], [1, 1])                     # unknown id: nothing changes
+    assert m.num_tokens(0) == 0 and m.num_free == 8
+    with pytest.raises(Exception):
+        m.append_batch([0], [-1])                          # negative count
+    slots, copies, cached = m.append_batch([], [])
+    assert len(slots) == 0 and copies == [] and cached == 0
+    slots, copies, _ = m.append_batch([0, 0], [3, 2])      # a sequence twice: appended in order
+    assert list(slots) == [0, 1, 2, 3, 4]                  # blocks 0 then 1 (default free order)
+    assert m.num_tokens(0) == 5
