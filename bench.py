@@ -465,6 +465,9 @@ def run_ours(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if ds.prefill else None
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(K)] if ds.prefill else None
+    # Decode: the timed steps run back to back with nothing between their kernels
+    # (an event between two kernels would cost the programmatic-launch overlap);
+    # the attend kernel alone is timed in a second pass with events around it.
     with ClockSampler(nvsmi_id(local), enabled=not args.no_clocks) as clocks:
         barrier()
         torch.cuda.synchronize()
@@ -473,14 +476,21 @@ def run_ours(args):
             if flush is not None:
                 flush.fill_(i & 0xFF)
                 ev_step[i][0].record(stream)
-            ds.run(ev_attend=ev[i])
+            ds.run(ev_attend=ev[i] if flush is not None else None)
             if flush is not None:
                 ev_step[i][1].record(stream)
         stop.record(stream)
         torch.cuda.synchronize()
         barrier()
     elapsed_ms = start.elapsed_time(stop) if flush is None else sum(a.elapsed_time(b) for a, b in ev_step)
-    attend_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    if flush is None:
+        n_att = min(K, 500)
+        for i in range(n_att):
+            ds.run(ev_attend=ev[i])
+        torch.cuda.synchronize()
+        attend_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev[:n_att])
+    else:
+        attend_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
     clock_info = clocks.summary()
 
     # end to end through the public API: host inputs in, host result out, every step
@@ -550,6 +560,8 @@ def run_ours(args):
             "frac": round(achieved_attend / peak, 4),
             "traffic": traffic,
             "attend_ms": round(attend_ms, 5),
+            "attend_timing": "CUDA events around each attend launch, in a pass after the timed steps "
+                             f"({min(K, 500)} launches)",
             "bytes_per_launch": alg_bytes,
         },
         "clocks": clock_info,
