@@ -316,14 +316,31 @@ class DeviceStep:
             self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
         self.tensor_core_prefill = self.prefill and pa.prefill_uses_tensor_cores(
             step.dtype, step.num_heads, step.num_kv_heads, step.head_dim, step.block_size)
-        # copy_blocks, reshape_and_cache, then plan/attend/reduce (decode), rows/plan/attend/reduce
-        # (prefill by decode rows) or plan/attend (tensor-core prefill)
-        body = 3 if not self.prefill else (2 if self.tensor_core_prefill else 4)
-        self.launches_per_step = (1 if len(step.copy_pairs) else 0) + 1 + body
+        # Decode: one pa_decode_step call -- copy_blocks (if any pairs), the prologue
+        # (plan + scatter of the new tokens), attend, reduce.  Prefill: copy_blocks,
+        # reshape_and_cache, then rows/plan/attend/reduce (prefill by decode rows) or
+        # plan/attend (tensor-core prefill).
+        copies = 1 if len(step.copy_pairs) else 0
+        if self.prefill:
+            self.launches_per_step = copies + 1 + (2 if self.tensor_core_prefill else 4)
+        else:
+            self.launches_per_step = copies + 3
 
     def run(self, ev_attend=None, q=None, new_key=None, new_value=None, slots=None, tables=None, ctx=None,
             out=None):
+        """One step.  A decode step without ``ev_attend`` is the single fused call
+        (pa_decode_step); with it, the same work runs phase by phase so that events
+        can bracket the attend kernel."""
         pa = self.pa
+        if not self.prefill and ev_attend is None:
+            pa.decode_step(out if out is not None else self.out, q if q is not None else self.q,
+                           new_key if new_key is not None else self.new_key,
+                           new_value if new_value is not None else self.new_value, self.kc, self.vc,
+                           slots if slots is not None else self.slots,
+                           tables if tables is not None else self.tables, ctx if ctx is not None else self.ctx,
+                           self.step.scale, copy_pairs=self.pairs if len(self.step.copy_pairs) else None,
+                           max_context_len=self.cap, partition_size=self.P, workspace=self.ws, dev_err=self.err)
+            return
         if len(self.step.copy_pairs):
             pa.copy_blocks(self.kc, self.vc, self.pairs, dev_err=self.err)
         pa.reshape_and_cache(new_key if new_key is not None else self.new_key,
@@ -548,6 +565,8 @@ def run_ours(args):
         "logical_bytes_per_step": logical_bytes,
         "effective_logical_gbs": round(logical_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
         "gpu_launches": ds.launches_per_step * K,
+        "step_call": "pa_decode_step: " + ("copy_blocks, " if len(step.copy_pairs) else "")
+                     + "plan+scatter prologue, attend, reduce",
         "kv_utilisation": kv_utilisation_summary(step, CONFIGS[args.config]["max_len"]),
         "roofline": {
             "kernel": "attend_bf16_kernel" if step.dtype == torch.bfloat16 else "attend_f32_kernel",

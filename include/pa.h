@@ -151,6 +151,28 @@ PA_API int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k
               int32_t* dev_err, pa_stream stream);
 
 /*
+ * pa_decode_step -- one whole decode step in one call: the copy-on-write block
+ * copies (pa_copy_blocks), the scatter of the step's new tokens
+ * (pa_reshape_and_cache) and pa_decode, with the same results as those three
+ * calls in that order.  The scatter and the decode's plan share one launch
+ * (neither reads what the other writes), so a step is at most four launches:
+ * copies (only when num_pairs > 0), scatter + plan, attention, merge.
+ *   key, value, slot_mapping, num_new_tokens   as for pa_reshape_and_cache
+ *                                             (the pool's shapes and dtype are
+ *                                             the decode's)
+ *   copy_pairs, num_pairs                      as for pa_copy_blocks
+ *   the rest                                   as for pa_decode
+ * Every argument of all three parts is checked before anything is launched.
+ */
+PA_API int pa_decode_step(void* out, pa_dtype out_dtype, const void* q, const void* key, const void* value,
+                          void* k_cache, void* v_cache, const int64_t* slot_mapping, int num_new_tokens,
+                          const int64_t* copy_pairs, int num_pairs, const int32_t* block_tables,
+                          const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                          int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                          int max_context_len, float scale, int partition_size, void* workspace,
+                          size_t workspace_bytes, pa_dtype dtype, int32_t* dev_err, pa_stream stream);
+
+/*
  * pa_decode_phases -- pa_decode split into its three launches, selected by the
  * bit mask `phases` (PA_PHASE_*; PA_PHASE_ALL gives pa_decode).  The plan
  * depends only on context_lens, the shapes and partition_size, so a caller

@@ -10,38 +10,15 @@
 
 #include "pa_device.cuh"
 #include "pa_host.h"
+#include "pa_scatter.cuh"
 
 namespace pa {
 
-// One CTA per new token.  A token's K (and V) for all kv heads is
-// num_kv_heads rows of `row_vecs` 16-byte vectors; row h goes to
-// cache[block][h][offset][:].
-__global__ void __launch_bounds__(256)
-reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
-                         uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
-                         const int64_t* __restrict__ slot_mapping, int num_kv_heads, int row_vecs,
-                         int block_size, int64_t num_slots, int32_t* dev_err) {
+// One CTA per new token (see scatter_token).
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(const ScatterArgs sa) {
     pdl_wait();
     pdl_launch_dependents();
-    const int t = blockIdx.x;
-    const int64_t slot = slot_mapping[t];
-    if (slot < 0) return;
-    if (slot >= num_slots) {
-        if (threadIdx.x == 0) flag_error(dev_err, PA_DEVERR_SLOT);
-        return;
-    }
-    const int64_t block = slot / block_size;
-    const int offset = static_cast<int>(slot - block * block_size);
-    const int per_token = num_kv_heads * row_vecs;
-    const uint4* ksrc = key + static_cast<int64_t>(t) * per_token;
-    const uint4* vsrc = value + static_cast<int64_t>(t) * per_token;
-    for (int i = threadIdx.x; i < per_token; i += blockDim.x) {
-        const int h = i / row_vecs;
-        const int v = i - h * row_vecs;
-        const int64_t dst = ((block * num_kv_heads + h) * block_size + offset) * row_vecs + v;
-        k_cache[dst] = ksrc[i];
-        v_cache[dst] = vsrc[i];
-    }
+    scatter_token(sa, static_cast<int>(blockIdx.x));
 }
 
 // grid.y = pair index; grid.x CTAs stride over the block's 16-byte vectors.
@@ -114,11 +91,19 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
     const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
     const int per_token = num_kv_heads * row_vecs;
     const int threads = per_token >= 256 ? 256 : ((per_token + 31) / 32) * 32;
+    ScatterArgs sa;
+    sa.key = static_cast<const uint4*>(key);
+    sa.value = static_cast<const uint4*>(value);
+    sa.k_cache = static_cast<uint4*>(k_cache);
+    sa.v_cache = static_cast<uint4*>(v_cache);
+    sa.slot_mapping = slot_mapping;
+    sa.num_kv_heads = num_kv_heads;
+    sa.row_vecs = row_vecs;
+    sa.block_size = block_size;
+    sa.num_slots = num_slots;
+    sa.dev_err = dev_err;
     return launch_status(launch_pdl(reshape_and_cache_kernel, dim3(num_tokens), dim3(threads), 0,
-                                    as_stream(stream), static_cast<const uint4*>(key),
-                                    static_cast<const uint4*>(value), static_cast<uint4*>(k_cache),
-                                    static_cast<uint4*>(v_cache), slot_mapping, num_kv_heads, row_vecs,
-                                    block_size, num_slots, dev_err));
+                                    as_stream(stream), sa));
 }
 
 extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,

@@ -44,6 +44,7 @@
 
 #include "pa_device.cuh"
 #include "pa_host.h"
+#include "pa_scatter.cuh"
 #include "pa_tma.h"
 #include "prefill_tc.h"
 
@@ -159,11 +160,10 @@ __device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, in
     return n;
 }
 
-__global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
+// The plan itself, run by one CTA of PLAN_THREADS threads.
+__device__ __forceinline__ void plan_body(const DecodeArgs& a) {
     __shared__ int scratch[33];
     __shared__ int lead[PLAN_THREADS];
-    pdl_wait();
-    pdl_launch_dependents();
     const int P = a.partition_size;
     // Sequences are taken PLAN_THREADS at a time (a multiple of every packing
     // run length).  Items: whole partitions first, then one per ragged tail,
@@ -231,6 +231,25 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
         base_tail += chunk_t;
     }
     if (threadIdx.x == 0) *a.ws_count = full_total + tail_total;
+}
+
+__global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
+    plan_body(a);
+}
+
+// One decode step's prologue in one launch: CTA 0 plans while CTAs 1..T write
+// the step's new tokens into the pool.  The plan reads only lengths and
+// tables, the scatter only the pool, so they need no order between them; the
+// attend kernel that follows waits for both.
+__global__ void __launch_bounds__(PLAN_THREADS) step_prologue_kernel(const DecodeArgs a, const ScatterArgs sa) {
+    pdl_wait();
+    pdl_launch_dependents();
+    if (blockIdx.x == 0)
+        plan_body(a);
+    else
+        scatter_token(sa, static_cast<int>(blockIdx.x) - 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -1001,7 +1020,7 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
                        int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
                        int partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
                        int32_t* dev_err, pa_stream stream, int phases, const int32_t* row_seq,
-                       Prep prep) {
+                       Prep prep, const ScatterArgs* scatter = nullptr, int num_new_tokens = 0) {
     // ---- host-side validation: nothing is launched unless everything is sane
     const int shape_rc = check_shapes(out_dtype, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                       num_blocks, max_blocks_per_seq, max_context_len, scale, partition_size,
@@ -1062,8 +1081,11 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
 
     if (prep(st, a.cap) != PA_OK) return PA_ERR_CUDA;
     if (phases & PA_PHASE_PLAN) {
-        if (launch_status(launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, st, a)) != PA_OK)
-            return PA_ERR_CUDA;
+        const cudaError_t e =
+            (scatter != nullptr && num_new_tokens > 0)
+                ? launch_pdl(step_prologue_kernel, dim3(1 + num_new_tokens), dim3(PLAN_THREADS), 0, st, a, *scatter)
+                : launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, st, a);
+        if (launch_status(e) != PA_OK) return PA_ERR_CUDA;
     }
     if (phases & PA_PHASE_ATTEND) {
         const long long unit_bound =
@@ -1181,6 +1203,48 @@ extern "C" int pa_prefill(void* out, pa_dtype out_dtype, const void* q, const vo
                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, max_context_len,
                        scale, partition_size, ws + rows, workspace_bytes - rows, dtype, dev_err, stream,
                        PA_PHASE_ALL, row_seq, prep);
+}
+
+extern "C" int pa_decode_step(void* out, pa_dtype out_dtype, const void* q, const void* key, const void* value,
+                              void* k_cache, void* v_cache, const int64_t* slot_mapping, int num_new_tokens,
+                              const int64_t* copy_pairs, int num_pairs, const int32_t* block_tables,
+                              const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                              int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                              int max_context_len, float scale, int partition_size, void* workspace,
+                              size_t workspace_bytes, pa_dtype dtype, int32_t* dev_err, pa_stream stream) {
+    // the scatter's and the copies' own checks; the decode's follow in decode_impl,
+    // and nothing launches before all of them pass
+    if (num_new_tokens < 0 || num_pairs < 0 || num_new_tokens > INT_MAX / 2) return PA_ERR_INVALID_ARG;
+    if (num_new_tokens > 0) {
+        if (!key || !value || !slot_mapping) return PA_ERR_INVALID_ARG;
+        if (!aligned_to(key, 16) || !aligned_to(value, 16) || !aligned_to(slot_mapping, 8))
+            return PA_ERR_INVALID_ARG;
+    }
+    if (num_pairs > 0 && (!copy_pairs || !aligned_to(copy_pairs, 8))) return PA_ERR_INVALID_ARG;
+    if (num_pairs > 65535) return PA_ERR_UNSUPPORTED;
+    if (!valid_dtype(dtype) || num_kv_heads <= 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    ScatterArgs sa;
+    sa.key = static_cast<const uint4*>(key);
+    sa.value = static_cast<const uint4*>(value);
+    sa.k_cache = static_cast<uint4*>(k_cache);
+    sa.v_cache = static_cast<uint4*>(v_cache);
+    sa.slot_mapping = slot_mapping;
+    sa.num_kv_heads = num_kv_heads;
+    sa.row_vecs = head_dim * element_bytes(dtype) / 16;
+    sa.block_size = block_size;
+    sa.num_slots = static_cast<int64_t>(num_blocks) * block_size;
+    sa.dev_err = dev_err;
+    const size_t block_bytes = static_cast<size_t>(num_kv_heads) * block_size * head_dim * element_bytes(dtype);
+    // copy-on-write copies first (the writes may land in the copied blocks)
+    auto copies = [=](cudaStream_t, int) {
+        return num_pairs > 0 ? pa_copy_blocks(k_cache, v_cache, copy_pairs, num_pairs, block_bytes, num_blocks,
+                                              dev_err, stream)
+                             : PA_OK;
+    };
+    return decode_impl(out, out_dtype, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+                       partition_size, workspace, workspace_bytes, dtype, dev_err, stream, PA_PHASE_ALL, nullptr,
+                       copies, &sa, num_new_tokens);
 }
 
 extern "C" int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,

@@ -34,6 +34,8 @@ SIGNATURES = {
     "pa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "pa_decode": (_i, _DECODE_ARGS),
     "pa_decode_phases": (_i, _DECODE_ARGS + [_i]),
+    "pa_decode_step": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i64p, _i, _i64p, _i, _i32p, _i32p, _i, _i, _i, _i,
+                            _i, _i, _i, _i, _f, _i, _vp, _sz, _i, _i32p, _vp]),
     "pa_copy_blocks": (_i, [_vp, _vp, _i64p, _i, _sz, _i, _i32p, _vp]),
     "pa_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "pa_prefill_uses_tensor_cores": (_i, [_i, _i, _i, _i, _i]),
@@ -185,6 +187,44 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), dtype_code(dt),
         _opt_err(dev_err), _stream_handle(stream), phases)
     _check(rc, "pa_decode")
+    return out
+
+
+def decode_step(out: torch.Tensor, q: torch.Tensor, key: torch.Tensor, value: torch.Tensor,
+                k_cache: torch.Tensor, v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, *,
+                copy_pairs: Optional[torch.Tensor] = None, max_context_len: int = 0, partition_size: int = 512,
+                workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One decode step in one call: copy-on-write copies (int64 [n][2]), the
+    scatter of key/value [T][Hkv][d] through slot_mapping, and paged decode
+    attention; writes and returns ``out`` [S][Hq][d]."""
+    NB, Hkv, B, d = k_cache.shape
+    S, Hq, dq = q.shape
+    T = key.shape[0]
+    if dq != d or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != (S, Hq, d):
+        raise ValueError("q / out must be [num_seqs][num_heads][head_dim] over the pool's head_dim")
+    if tuple(key.shape) != (T, Hkv, d) or tuple(value.shape) != (T, Hkv, d) or tuple(slot_mapping.shape) != (T,):
+        raise ValueError("key/value must be [T][num_kv_heads][head_dim] and slot_mapping [T]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [num_seqs][max_blocks] and context_lens [num_seqs]")
+    npairs = 0 if copy_pairs is None else int(copy_pairs.shape[0])
+    if npairs and (copy_pairs.dim() != 2 or copy_pairs.shape[1] != 2):
+        raise ValueError("copy_pairs must be int64 [n][2]")
+    dt = k_cache.dtype
+    if workspace is None:
+        cap = decode_capacity(block_tables, B, max_context_len)
+        workspace = alloc_workspace(S, Hq, d, cap, partition_size, q.device)
+    rc = lib.pa_decode_step(
+        _dev(out, "out"), dtype_code(out.dtype), _dev(q, "q", dt), _dev(key, "key", dt) if T else None,
+        _dev(value, "value", dt) if T else None, _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(slot_mapping, "slot_mapping", torch.int64) if T else None, T,
+        _dev(copy_pairs, "copy_pairs", torch.int64) if npairs else None, npairs,
+        _dev(block_tables, "block_tables", torch.int32), _dev(context_lens, "context_lens", torch.int32), S, Hq,
+        Hkv, d, B, NB, block_tables.shape[1], max_context_len, float(scale), partition_size,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), dtype_code(dt), _opt_err(dev_err),
+        _stream_handle(stream))
+    _check(rc, "pa_decode_step")
     return out
 
 

@@ -426,6 +426,35 @@ def test_random_fork_histories(pa, seed, heads):
         assert torch.equal(out, out2)
 
 
+@pytest.mark.parametrize("name", ["independent", "cow", "poisoned", "no_new_tokens"])
+def test_decode_step_equals_the_three_calls(pa, name):
+    """pa_decode_step (copies, scatter fused with the plan, attention, merge) gives
+    bit for bit the pools and output of pa_copy_blocks, pa_reshape_and_cache and
+    pa_decode called in that order."""
+    kw = dict(num_heads=32, num_kv_heads=8, head_dim=128, block_size=16, partition_size=64, device="cuda")
+    if name == "cow":
+        step = W.shared_prefix(prompt_len=40, suffix_max=0, prompts=3, samples=4, **kw)
+    else:
+        step = to_device(W.independent(name, [5, 70, 300, 1, 129, 1000], dtype=torch.bfloat16, seed=12,
+                                       poison=(name == "poisoned"), **{k: v for k, v in kw.items()
+                                                                        if k != "device"}))
+    slots = step.slot_mapping if name != "no_new_tokens" else np.zeros(0, dtype=np.int64)
+    ref_out, ref_k, ref_v, ref_err, _ = run_gpu(pa, step, slots=slots)
+    kc, vc = step.k_cache.clone(), step.v_cache.clone()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(ref_out)
+    T = len(slots)
+    pairs = torch.from_numpy(np.ascontiguousarray(step.copy_pairs)).cuda() if len(step.copy_pairs) else None
+    pa.decode_step(out, step.q, step.new_key[:T], step.new_value[:T], kc, vc, torch.from_numpy(slots).cuda(),
+                   torch.from_numpy(step.block_tables).cuda(), torch.from_numpy(step.context_lens).cuda(), step.scale,
+                   copy_pairs=pairs, partition_size=step.partition_size, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == ref_err
+    assert torch.equal(out, ref_out)
+    assert torch.equal(kc.view(torch.int16), ref_k.view(torch.int16))
+    assert torch.equal(vc.view(torch.int16), ref_v.view(torch.int16))
+
+
 def test_bounded_wait_gives_up_and_the_context_survives(pa):
     """The bounded wait all asynchronous-copy waits use: a barrier nothing arrives
     at is given up on after the limit, PA_DEVERR_TIMEOUT is raised, the kernel

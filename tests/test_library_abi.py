@@ -55,6 +55,28 @@ def test_status_strings_and_version(pa):
     assert pa.lib.pa_version() >= 100
 
 
+def test_decode_step_host_validation(pa):
+    """pa_decode_step refuses bad scatter, copy or decode arguments before any
+    launch (no GPU needed)."""
+    f = pa.lib.pa_decode_step
+    base = dict(out=256, od=pa.PA_F32, q=256, key=256, value=256, k=256, v=256, slots=256, T=4, pairs=None,
+                npairs=0, tables=256, ctx=256, S=4, Hq=32, Hkv=8, d=128, B=16, NB=64, mb=8, maxc=0, scale=0.1,
+                P=512, ws=None, wsb=0, dt=pa.PA_BF16, err=None, st=None)
+
+    def call(**over):
+        a = {**base, **over}
+        return f(a["out"], a["od"], a["q"], a["key"], a["value"], a["k"], a["v"], a["slots"], a["T"], a["pairs"],
+                 a["npairs"], a["tables"], a["ctx"], a["S"], a["Hq"], a["Hkv"], a["d"], a["B"], a["NB"], a["mb"],
+                 a["maxc"], a["scale"], a["P"], a["ws"], a["wsb"], a["dt"], a["err"], a["st"])
+
+    assert call(key=None) == pa.PA_ERR_INVALID_ARG              # new tokens without keys
+    assert call(slots=258) == pa.PA_ERR_INVALID_ARG             # misaligned slot mapping
+    assert call(npairs=2) == pa.PA_ERR_INVALID_ARG              # pairs announced, none given
+    assert call(T=-1) == pa.PA_ERR_INVALID_ARG
+    assert call(d=96) == pa.PA_ERR_UNSUPPORTED                  # the decode's own checks
+    assert call(ws=None, wsb=0) == pa.PA_ERR_INVALID_ARG        # no workspace
+
+
 def test_selftest_host_validation(pa):
     """Bad arguments of the bounded-wait self-test are refused before any launch."""
     f = pa.lib.pa_selftest_bounded_wait
