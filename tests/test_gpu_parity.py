@@ -253,10 +253,36 @@ FULL = {
 }
 
 
+def run_fused_step(pa, step, out_dtype):
+    """The benchmark's launch configuration: one pa_decode_step call with the
+    capacity bound, workspace and output dtype bench.py uses."""
+    dev = "cuda"
+    pre = (step.k_cache.clone(), step.v_cache.clone())
+    kc, vc = step.k_cache.clone(), step.v_cache.clone()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    tables = torch.from_numpy(step.block_tables.astype(np.int32)).to(dev)
+    cap = pa.decode_capacity(tables, step.block_size, step.max_context_len)
+    ws = pa.alloc_workspace(step.num_seqs, step.num_heads, step.head_dim, cap, step.partition_size, dev)
+    out = torch.empty(step.num_seqs, step.num_heads, step.head_dim, dtype=out_dtype, device=dev)
+    pairs = torch.from_numpy(np.ascontiguousarray(step.copy_pairs)).to(dev) if len(step.copy_pairs) else None
+    pa.decode_step(out, step.q, step.new_key, step.new_value, kc, vc, torch.from_numpy(step.slot_mapping).to(dev),
+                   tables, torch.from_numpy(step.context_lens.astype(np.int32)).to(dev), step.scale,
+                   copy_pairs=pairs, max_context_len=cap, partition_size=step.partition_size, workspace=ws,
+                   dev_err=err)
+    torch.cuda.synchronize()
+    return out, kc, vc, int(err.item()), pre
+
+
+@pytest.mark.parametrize("call", ["phased", "fused_step_bf16_out"])
 @pytest.mark.parametrize("name", list(FULL))
-def test_full_size(pa, name):
+def test_full_size(pa, name, call):
     step = FULL[name]()
-    out, kc, vc, err, pre = run_gpu(pa, step, keep_pre=True)
+    if call == "phased":
+        out_dtype = torch.float32
+        out, kc, vc, err, pre = run_gpu(pa, step, keep_pre=True)
+    else:
+        out_dtype = torch.bfloat16
+        out, kc, vc, err, pre = run_fused_step(pa, step, out_dtype)
     assert err == 0
     assert torch.isfinite(out).all()
     pre_k, pre_v = pre
@@ -284,7 +310,7 @@ def test_full_size(pa, name):
     ref = oracle_outputs(step, seqs, pre_k, pre_v)
     got = f64(out)
     for s in seqs:
-        assert_close(got[s], ref[s], torch.bfloat16, torch.float32, f"{name} seq {s} ctx {ctx[s]}")
+        assert_close(got[s], ref[s], torch.bfloat16, out_dtype, f"{name} seq {s} ctx {ctx[s]}")
 
 
 # ---------------------------------------------------------------------------
