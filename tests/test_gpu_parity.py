@@ -362,6 +362,28 @@ def test_deterministic_and_shared_tables(pa):
     assert torch.equal(a[0], a[1])
 
 
+def test_attend_phases_repeat_over_one_plan(pa):
+    """Units are handed out by a ticket that the plan resets and the last attend
+    CTA puts back: attend + reduce run twice over one plan give the result of
+    the whole call, bit for bit, both times (many more units than CTAs)."""
+    step = to_device(W.independent("phases", [2000] * 96 + [17] * 64, dtype=torch.bfloat16, num_heads=32,
+                                   num_kv_heads=8, head_dim=128, block_size=16, seed=8, partition_size=128))
+    ref, kc, vc, err, _ = run_gpu(pa, step)
+    assert err == 0
+    tables = torch.from_numpy(step.block_tables.astype(np.int32)).cuda()
+    ctx = torch.from_numpy(step.context_lens.astype(np.int32)).cuda()
+    ws = pa.alloc_workspace(step.num_seqs, step.num_heads, step.head_dim,
+                            pa.decode_capacity(tables, step.block_size, 0), step.partition_size, "cuda")
+    kw = dict(partition_size=step.partition_size, workspace=ws)
+    pa.decode(torch.empty_like(ref), step.q, kc, vc, tables, ctx, step.scale, phases=pa.PHASE_PLAN, **kw)
+    for _ in range(2):
+        out = torch.full_like(ref, float("nan"))
+        pa.decode(out, step.q, kc, vc, tables, ctx, step.scale, phases=pa.PHASE_ATTEND, **kw)
+        pa.decode(out, step.q, kc, vc, tables, ctx, step.scale, phases=pa.PHASE_REDUCE, **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+
+
 def unshared_copy(step):
     """The same batch with every sequence's blocks copied to private physical
     blocks: identical contents, no shared block ids, hence no packed units."""
