@@ -179,7 +179,9 @@ PA_API int pa_decode_step(void* out, pa_dtype out_dtype, const void* q, const vo
  * running several layers over the same batch may plan once and run
  * ATTEND|REDUCE per layer with the same workspace; a caller timing the
  * attention kernel alone brackets the ATTEND call with its own events.
- * Phases must run in order PLAN, ATTEND, REDUCE on the same workspace.
+ * Phases must run in order PLAN, ATTEND, REDUCE on the same workspace, and two
+ * ATTEND launches over one workspace must not overlap in time: they share its
+ * unit counter, which each ATTEND leaves as the plan left it.
  * Arguments as for pa_decode.
  */
 #define PA_PHASE_PLAN   0x1
