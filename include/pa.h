@@ -181,7 +181,8 @@ PA_API int pa_decode_step(void* out, pa_dtype out_dtype, const void* q, const vo
  * attention kernel alone brackets the ATTEND call with its own events.
  * Phases must run in order PLAN, ATTEND, REDUCE on the same workspace, and two
  * ATTEND launches over one workspace must not overlap in time: they share its
- * unit counter, which each ATTEND leaves as the plan left it.
+ * unit counter, which each completed ATTEND leaves as the plan left it (after
+ * a PA_DEVERR_TIMEOUT, plan again).
  * Arguments as for pa_decode.
  */
 #define PA_PHASE_PLAN   0x1

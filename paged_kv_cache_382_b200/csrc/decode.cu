@@ -60,8 +60,8 @@ struct DecodeArgs {
     const int32_t* context_lens;
     int32_t* dev_err;
     int* ws_count;       // [1]   number of work items
-    unsigned long long* ws_ticket;   // [1] bf16 attend: units taken past the first grid-wide wave (0 after the plan)
-    unsigned int* ws_done;           // [1] attend CTAs finished (the last one sets both back to 0)
+    unsigned long long* ws_ticket;   // [1] bf16 attend: units taken past the first grid-wide wave (0 after
+                                     //     the plan; the last fetch of a launch sets it back to 0)
     int* ws_items;       // [num_seqs * max_parts]  see make_item
     float2* ws_ml;       // [num_seqs][num_heads][max_parts]  (log2-domain max, sum)
     float* ws_acc;       // [num_seqs][num_heads][max_parts][head_dim]
@@ -166,10 +166,7 @@ __device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, in
 __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
     __shared__ int scratch[33];
     __shared__ int lead[PLAN_THREADS];
-    if (threadIdx.x == 0) {
-        *a.ws_ticket = 0;
-        *a.ws_done = 0;
-    }
+    if (threadIdx.x == 0) *a.ws_ticket = 0;
     const int P = a.partition_size;
     // Sequences are taken PLAN_THREADS at a time (a multiple of every packing
     // run length).  Items: whole partitions first, then one per ragged tail,
@@ -424,7 +421,13 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
         __syncthreads();   // the previous unit's epilogue is done with shared memory; s_next read
         if (s_abort) break;
-        if (tid == 0) s_next = gridDim.x + atomicAdd(a.ws_ticket, 1ull);   // the CTA's next unit
+        if (tid == 0) {   // the CTA's next unit
+            // One fetch per unit run, so fetch number units - 1 is the launch's
+            // last: it puts the ticket back for another launch over this plan.
+            const unsigned long long v = atomicAdd(a.ws_ticket, 1ull);
+            if (v + 1 == static_cast<unsigned long long>(units)) *a.ws_ticket = 0ull;
+            s_next = gridDim.x + v;
+        }
         if (tid < 8) {
             int member, head;
             bool valid;
@@ -640,16 +643,6 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         __syncthreads();
         combine_store<W, D>(a, mm, ml, mo, s_rows, p, nrows);
         fence_proxy_async_smem();   // these generic accesses precede the next unit's bulk copies
-    }
-    // The last CTA to finish sets the ticket back to 0, so that another launch
-    // over the same plan (an attend-only call) sees every unit again.  Every
-    // CTA has taken its last ticket before it counts itself done.
-    if (tid == 0) {
-        __threadfence();
-        if (atomicAdd(a.ws_done, 1u) == gridDim.x - 1) {
-            *a.ws_ticket = 0ull;
-            *a.ws_done = 0u;
-        }
     }
 }
 
@@ -940,7 +933,7 @@ struct WsLayout {
 
 inline WsLayout ws_layout(int S, int Hq, int D, int max_parts) {
     WsLayout L;
-    size_t off = 256;   // header: the work-item count (0), the attend ticket (8) and done count (16)
+    size_t off = 256;   // header: the work-item count (0) and the attend kernel's unit ticket (8)
     L.items = off;
     off += round_up(static_cast<size_t>(S) * max_parts * sizeof(int), 256);
     if (max_parts > 1) {
@@ -1083,7 +1076,6 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     a.ws_count = reinterpret_cast<int*>(ws);
     a.ws_ticket = reinterpret_cast<unsigned long long*>(ws + 8);
-    a.ws_done = reinterpret_cast<unsigned int*>(ws + 16);
     a.ws_items = reinterpret_cast<int*>(ws + L.items);
     a.ws_ml = max_parts > 1 ? reinterpret_cast<float2*>(ws + L.ml) : nullptr;
     a.ws_acc = max_parts > 1 ? reinterpret_cast<float*>(ws + L.acc) : nullptr;

@@ -363,9 +363,10 @@ def test_deterministic_and_shared_tables(pa):
 
 
 def test_attend_phases_repeat_over_one_plan(pa):
-    """Units are handed out by a ticket that the plan resets and the last attend
-    CTA puts back: attend + reduce run twice over one plan give the result of
-    the whole call, bit for bit, both times (many more units than CTAs)."""
+    """Units are handed out by a ticket that the plan resets and each attend
+    launch's last fetch puts back: attend + reduce run twice over one plan give
+    the result of the whole call, bit for bit, both times (many more units
+    than CTAs)."""
     step = to_device(W.independent("phases", [2000] * 96 + [17] * 64, dtype=torch.bfloat16, num_heads=32,
                                    num_kv_heads=8, head_dim=128, block_size=16, seed=8, partition_size=128))
     ref, kc, vc, err, _ = run_gpu(pa, step)
