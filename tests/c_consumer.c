@@ -38,6 +38,11 @@ int main(void) {
                     NULL, 0, PA_BF16, NULL, NULL) == PA_ERR_INVALID_ARG);
     CHECK(pa_decode(NULL, PA_F32, NULL, NULL, NULL, NULL, NULL, 1, 32, 8, 96, 16, 64, 4, 0, 0.1f, 512,
                     NULL, 0, PA_BF16, NULL, NULL) == PA_ERR_UNSUPPORTED);   /* head_dim 96 */
+    /* the one-call step checks its scatter, copy and decode arguments first */
+    CHECK(pa_decode_step(NULL, PA_F32, NULL, NULL, NULL, NULL, NULL, NULL, 4, NULL, 0, NULL, NULL, 1, 32, 8,
+                         128, 16, 64, 4, 0, 0.1f, 512, NULL, 0, PA_BF16, NULL, NULL) == PA_ERR_INVALID_ARG);
+    CHECK(pa_decode_step(NULL, PA_F32, NULL, NULL, NULL, NULL, NULL, NULL, -1, NULL, 0, NULL, NULL, 1, 32, 8,
+                         128, 16, 64, 4, 0, 0.1f, 512, NULL, 0, PA_BF16, NULL, NULL) == PA_ERR_INVALID_ARG);
     CHECK(pa_reshape_and_cache(NULL, NULL, NULL, NULL, NULL, 1, 8, 128, 16, 64, PA_BF16, NULL, NULL) ==
           PA_ERR_INVALID_ARG);
     CHECK(pa_copy_blocks(NULL, NULL, NULL, 0, 16, 4, NULL, NULL) == PA_OK);       /* no pairs: no-op */
