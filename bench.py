@@ -821,10 +821,11 @@ def run_block_manager(args):
             for r in range(R):
                 m.append(r, one if cache else 1)
         t2 = time.perf_counter()
-        ids = list(range(R))
-        batch = [one] * R if cache else [1] * R
-        for _ in range(STEPS - half):              # one call per step (pa_bm_append_batch)
-            m.append_batch(ids, batch)
+        ids = np.arange(R, dtype=np.int64)
+        counts = np.ones(R, dtype=np.int32)
+        step_tokens = np.zeros(R, dtype=np.int32) if cache else None
+        for _ in range(STEPS - half):              # one call per step (pa_bm_append_batch), flat arrays
+            m.append_batch(ids, step_tokens, counts=counts)
         t3 = time.perf_counter()
         key = "prefix_cache" if cache else "no_cache"
         res[key] = {"admit_tokens_per_s": round(R * (P_SYS + USER) / (t1 - t0), 1),
@@ -839,7 +840,8 @@ def run_block_manager(args):
             "config": {"workload": CONFIGS["host_block_manager"]["desc"], "name": "host_block_manager"},
             "results": res,
             "note": "timed through the Python binding: one ctypes call per request for admission; decode "
-                    "appends one call per sequence and step, then one pa_bm_append_batch call per step"}
+                    "appends one call per sequence and step, then one pa_bm_append_batch call per step "
+                    "over flat id / count / token arrays"}
     print(json.dumps(line), flush=True)
 
 

@@ -366,13 +366,20 @@ class NativeBlockManager:
         pairs = [(int(copies[2 * i]), int(copies[2 * i + 1])) for i in range(ncopies.value)]
         return slots[:n], pairs, ncached.value
 
-    def append_batch(self, seq_ids, tokens, max_copies=None):
+    def append_batch(self, seq_ids, tokens, max_copies=None, counts=None):
         """One call for a batch: tokens[k] (a count, or token ids when prefix
-        caching) appended to seq_ids[k].  Returns (slots of all new tokens in
-        order, [(src, dst) copies], tokens served from the cache)."""
+        caching) appended to seq_ids[k].  With `counts` given, `tokens` is
+        instead one flat array of all the token ids in order (or None without
+        prefix caching), as a serving loop holds them.  Returns (slots of all
+        new tokens in order, [(src, dst) copies], tokens served from the cache)."""
         np = self._np
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
-        if all(isinstance(t, (int, np.integer)) for t in tokens):
+        if counts is not None:
+            counts = np.ascontiguousarray(counts, dtype=np.int32)
+            toks = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+            if toks is not None and toks.size != int(counts.sum()):
+                raise ValueError("tokens must hold sum(counts) token ids")
+        elif all(isinstance(t, (int, np.integer)) for t in tokens):
             counts = np.ascontiguousarray(tokens, dtype=np.int32)
             toks = None
         else:

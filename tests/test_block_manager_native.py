@@ -183,7 +183,13 @@ def test_append_batch_equals_one_call_per_sequence(pa, prefix_cache):
             want_slots += list(s)
             want_copies += c
             want_cached += k
-        got_slots, got_copies, got_cached = b.append_batch(seqs, batch if prefix_cache else [len(t) for t in batch])
+        if step % 2 == 0:
+            got_slots, got_copies, got_cached = b.append_batch(seqs, batch if prefix_cache
+                                                               else [len(t) for t in batch])
+        else:                                              # flat arrays, as a serving loop holds them
+            flat = np.concatenate([np.asarray(t, dtype=np.int32) for t in batch]) if prefix_cache else None
+            got_slots, got_copies, got_cached = b.append_batch(np.asarray(seqs), flat,
+                                                               counts=[len(t) for t in batch])
         assert list(got_slots) == want_slots and got_copies == want_copies and got_cached == want_cached
     for sid in seqs:
         assert a.block_table(sid) == b.block_table(sid)
@@ -198,6 +204,8 @@ def test_append_batch_validation(pa):
     assert m.num_tokens(0) == 0 and m.num_free == 8
     with pytest.raises(Exception):
         m.append_batch([0], [-1])                          # negative count
+    with pytest.raises(ValueError):
+        pa.NativeBlockManager(8, 4, prefix_cache=True).append_batch([0], np.zeros(3, np.int32), counts=[2])
     slots, copies, cached = m.append_batch([], [])
     assert len(slots) == 0 and copies == [] and cached == 0
     slots, copies, _ = m.append_batch([0, 0], [3, 2])      # a sequence twice: appended in order
