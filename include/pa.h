@@ -339,8 +339,6 @@ PA_API int pa_bm_free(pa_block_manager* manager, int64_t seq_id);
 PA_API int pa_bm_append(pa_block_manager* manager, int64_t seq_id, const int32_t* token_ids,
                         int num_tokens, int64_t* slots, int64_t* copies, int max_copies,
                         int* num_copies, int* num_cached_tokens);
-/* The sequence's block table (out may be NULL to query *num_blocks); PA_ERR_WORKSPACE if
- * it has more than max_blocks entries.  *num_tokens (nullable) gets its length. */
 /*
  * pa_bm_append_batch -- pa_bm_append for many sequences in one call (one decode
  * step of a batch: num_seqs sequences, counts[k] tokens for seq_ids[k]).
@@ -355,6 +353,8 @@ PA_API int pa_bm_append(pa_block_manager* manager, int64_t seq_id, const int32_t
 PA_API int pa_bm_append_batch(pa_block_manager* manager, int num_seqs, const int64_t* seq_ids,
                               const int32_t* counts, const int32_t* token_ids, int64_t* slots,
                               int64_t* copies, int max_copies, int* num_copies, int* num_cached_tokens);
+/* The sequence's block table (out may be NULL to query *num_blocks); PA_ERR_WORKSPACE if
+ * it has more than max_blocks entries.  *num_tokens (nullable) gets its length. */
 PA_API int pa_bm_block_table(const pa_block_manager* manager, int64_t seq_id, int32_t* out,
                              int max_blocks, int* num_blocks, int64_t* num_tokens);
 PA_API int pa_bm_num_free(const pa_block_manager* manager);
