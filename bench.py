@@ -13,14 +13,20 @@ Metric: paged decode attention KV GB/s (algorithmic bytes / step time; also as
   sum_s ctx_s*Hkv*d*2*e + 2*S*Hq*d*e + sum_s ceil(ctx_s/B)*4 + 4*S
 (shared prefix blocks counted once).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME|decode] [--impl ours|reference]
 
-Default workload: Llama-7B-like decode layer in bf16 (64 sequences, 32 = 32
-heads, head_dim 128, block_size 16, context lengths uniform [128, 2048], an
-8192-block pool popped from a shuffled free list) plus the scatter of 64 new
-tokens.  Its K/V (1.16 GB per step) is far larger than the 126 MB L2, so no L2
-flush is needed between steps.  With N > 1 ranks (torchrun) every rank runs its
-own batch (seed + rank): weak scaling, no collective on the data path.
+Default (--config decode): every decode workload in one run.  The JSON line's
+headline is the GQA batch (256 sequences, 32 q / 8 kv heads, head_dim 128,
+block_size 16, log-normal context lengths with median 1000, a 90 % occupied
+pool), the largest batch of the suite, timed over exactly K steps; its
+``per_config`` object holds the same measurements for every decode workload:
+Llama-7B-like, GQA, parallel sampling with a shared 512-token prompt (and the
+520-token prompt's copy-on-write step) and long context at block size 8, 16
+and 32.  Workloads whose unique bytes are under twice the 126 MB L2 have L2
+flushed (a 256 MB write) before every timed step, outside per-step CUDA
+events; the others are larger than L2 and run back to back.  With N > 1 ranks
+(torchrun) every rank runs its own batches (seed + rank): weak scaling, no
+collective on the data path.
 
 Rank 0 prints one JSON line.
 """
@@ -79,7 +85,14 @@ CONFIGS["host_block_manager"] = dict(
     max_len=0, builder=None, kwargs={},
     desc="host block manager (pa_bm_*, C++): 256 requests with a 512-token shared system prompt + "
          "64 user tokens, then 256 decode steps of one token each, block_size 16")
-DEFAULT_CONFIG = "llama7b"
+DECODE_SUITE = ["llama7b", "gqa", "shared_prefix", "shared_prefix_cow", "long_context_b8", "long_context_b16",
+                "long_context_b32"]
+SUITE_HEADLINE = "gqa"
+DEFAULT_CONFIG = "decode"
+L2_BYTES = 126 * 1024 * 1024
+# per-config entries other than the headline run enough steps to fill this much
+# device time (at least K), so that short steps are not timed over a few ms only
+PER_CONFIG_MIN_SECONDS = 0.25
 # sources that make up each profiled kernel: a committed ncu summary counts only
 # while their hash is the one it records
 KERNEL_SOURCES = {
@@ -95,9 +108,10 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=5000)
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--config", choices=sorted(CONFIGS), default=DEFAULT_CONFIG)
+    p.add_argument("--config", choices=sorted(CONFIGS) + [DEFAULT_CONFIG], default=DEFAULT_CONFIG)
     p.add_argument("--seed", type=int, default=0)
-    p.add_argument("--partition-size", type=int, default=512)
+    p.add_argument("--partition-size", type=int, default=None,
+                   help="tokens per split-context partition (default: the workload's own, 512 unless stated)")
     p.add_argument("--cpu-core-seconds", type=float, default=15.0,
                    help="CPU work of the oracle baseline sample, in core-seconds")
     p.add_argument("--reference-seconds", type=float, default=150.0,
@@ -105,6 +119,10 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-flush", action="store_true",
+                   help="run every workload's steps back to back, without L2 flushes (comparisons only)")
+    p.add_argument("--eager", action="store_true",
+                   help="time eager pa_decode_step calls instead of replays of captured CUDA graphs")
     return p.parse_args(argv)
 
 
@@ -326,6 +344,18 @@ class DeviceStep:
         else:
             self.launches_per_step = copies + 3
 
+    def capture(self, n):
+        """A CUDA graph of n consecutive decode steps (one pa_decode_step call each,
+        on these buffers), as a serving loop replays its decode step: the same
+        kernels and work as eager calls, without the host's per-call cost."""
+        import torch
+
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            for _ in range(n):
+                self.run()
+        return g
+
     def run(self, ev_attend=None, q=None, new_key=None, new_value=None, slots=None, tables=None, ctx=None,
             out=None):
         """One step.  A decode step without ``ev_attend`` is the single fused call
@@ -387,6 +417,11 @@ def kv_utilisation_summary(step, max_len):
             "block_size": u["block_size"], "max_len": u["max_len"]}
 
 
+def partition_for(args, config: str) -> int:
+    """The partition size a workload runs with: --partition-size if given, else its own."""
+    return args.partition_size or CONFIGS[config].get("partition_size", 512)
+
+
 def build_step(config: str, seed: int, device, partition_size: int):
     from paged_kv_cache_382_b200 import workloads as W
 
@@ -437,12 +472,219 @@ def barrier():
         dist.barrier()
 
 
+def config_dict(name, step, world, partition_size, flushed):
+    """The line's ``config`` (the same keys in both arms)."""
+    from paged_kv_cache_382_b200 import workloads as W
+
+    alg = W.algorithmic_bytes(step, unique=True)
+    if flushed:
+        l2 = (f"L2 flushed before every timed step (a 256 MB write outside the per-step CUDA events): "
+              f"{alg / 1e6:.1f} MB of unique K/V+q/out per step is under twice the 126 MB L2")
+    else:
+        l2 = f"inputs larger than L2: {alg / 1e9:.3f} GB of K/V+q/out per step vs 126 MB L2, steps back to back"
+    return {
+        "workload": CONFIGS[name]["desc"],
+        "name": name,
+        "num_seqs_per_gpu": step.num_seqs,
+        "context_tokens_per_gpu": int(step.context_lens.sum()),
+        "partition_size": partition_size,
+        "parallelism": f"replicas x{world} (independent batches, no collective)",
+        "l2": l2,
+    }
+
+
+def needs_flush(step) -> bool:
+    from paged_kv_cache_382_b200 import workloads as W
+
+    return W.algorithmic_bytes(step, unique=True) < 2 * L2_BYTES
+
+
+GRAPH_CHUNK = 16   # steps per replayed CUDA graph when steps run back to back
+
+
+class StepGraphs:
+    """CUDA graphs of 1 and GRAPH_CHUNK decode steps; n steps replay
+    n // GRAPH_CHUNK large graphs and n % GRAPH_CHUNK small ones."""
+
+    def __init__(self, ds, warmup):
+        import torch
+
+        self.one = ds.capture(1)
+        self.chunk = ds.capture(GRAPH_CHUNK)
+        for _ in range(max(warmup, 1)):
+            self.one.replay()
+            self.chunk.replay()
+        torch.cuda.synchronize()
+
+    def replay(self, n):
+        for _ in range(n // GRAPH_CHUNK):
+            self.chunk.replay()
+        for _ in range(n % GRAPH_CHUNK):
+            self.one.replay()
+
+
+def time_steps(ds, n, flush, stream, graphs=None):
+    """Device time (ms) of n steps, and the host time (ms) spent enqueueing them:
+    back to back between two events, or, with a flush buffer, each step between
+    its own events after an L2 flush.  With ``graphs`` the steps are replays of
+    captured CUDA graphs, otherwise eager pa_decode_step calls."""
+    import torch
+
+    if flush is None:
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        start.record(stream)
+        if graphs is not None:
+            graphs.replay(n)
+        else:
+            for _ in range(n):
+                ds.run()
+        stop.record(stream)
+        host_ms = (time.perf_counter() - t0) * 1e3
+        torch.cuda.synchronize()
+        return start.elapsed_time(stop), host_ms
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    t0 = time.perf_counter()
+    for i in range(n):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        if graphs is not None:
+            graphs.one.replay()
+        else:
+            ds.run()
+        ev[i][1].record(stream)
+    host_ms = (time.perf_counter() - t0) * 1e3
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev), host_ms
+
+
+def time_attend(ds, n, flush):
+    """Mean device time (ms) of the attend kernel alone: the step runs phase by
+    phase with events around the attend launch (after an L2 flush if given)."""
+    import torch
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        ds.run(ev_attend=ev[i])
+    torch.cuda.synchronize()
+    return statistics.fmean(a.elapsed_time(b) for a, b in ev)
+
+
+def measure_decode(pa, args, name, dev, world, rank, local, steps, warmup, pool=None, cores=None):
+    """Every measurement of one decode workload; ``steps`` None picks a count that
+    fills PER_CONFIG_MIN_SECONDS of device time (at least --steps)."""
+    import torch
+
+    from paged_kv_cache_382_b200 import workloads as W
+
+    P = partition_for(args, name)
+    step = build_step(name, args.seed + rank, dev, P)
+    ds = DeviceStep(pa, step, P)
+    alg_bytes = W.algorithmic_bytes(step, unique=True)
+    logical_bytes = W.algorithmic_bytes(step, unique=False)
+    ctx_tokens = int(step.context_lens.sum())
+    flush = (torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+             if needs_flush(step) and not args.no_flush else None)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        ds.run()
+    torch.cuda.synchronize()
+    if int(ds.err.item()) != 0:
+        raise RuntimeError(f"{name}: device error word {int(ds.err.item()):#x}")
+    graphs = None if args.eager else StepGraphs(ds, warmup)
+    if steps is None:
+        est = time_steps(ds, 5, flush, stream, graphs)[0] / 5
+        want = int(math.ceil(PER_CONFIG_MIN_SECONDS * 1e3 / max(est, 1e-4)))
+        steps = int(reduce_over_ranks([min(5000, max(args.steps, want))], ["max"])[0])
+    K = steps
+    with ClockSampler(nvsmi_id(local), enabled=not args.no_clocks) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        elapsed_ms, host_ms = time_steps(ds, K, flush, stream, graphs)
+        torch.cuda.synchronize()
+        barrier()
+    # the same steps as eager calls (host-side cost per step included), for reference
+    eager_ms, eager_host_ms = time_steps(ds, K, flush, stream) if graphs is not None else (elapsed_ms, host_ms)
+    n_att = min(K, 500)
+    attend_ms = time_attend(ds, n_att, flush)
+    clock_info = clocks.summary()
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(ds, step, alg_bytes, warmup, min(K, 1000), flush)
+    tot_bytes, max_ms, tot_tokens, tot_seqs = reduce_over_ranks(
+        [alg_bytes * K, elapsed_ms, ctx_tokens * K, step.num_seqs * K], ["sum", "max", "sum", "sum"])
+    e2e_line = None
+    if e2e is not None:
+        e2e_bytes, e2e_ms = reduce_over_ranks([e2e["bytes"], e2e["ms"]], ["sum", "max"])
+        e2e_line = {"value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "ms_per_step": round(e2e_ms / e2e["steps"], 5), "steps": e2e["steps"],
+                    "timing": e2e["timing"]}
+    peak, peak_kind = measured_hbm_peak()
+    achieved_attend = alg_bytes / (attend_ms * 1e-3) / 1e9
+    value = tot_bytes / (max_ms * 1e-3) / 1e9
+    traffic = profiled_traffic(name)
+    cpu = None
+    if pool is not None:
+        cpu = cpu_baseline(step, pool, cores, args.cpu_core_seconds)
+    res = {
+        "value": round(value, 2),
+        "unit": UNIT,
+        "steps": K,
+        "ms_per_step": round(max_ms / K, 5),
+        "config": config_dict(name, step, world, P, flush is not None),
+        "pct_of_8tbs": round(100.0 * value / NOMINAL_HBM_GBS, 2),
+        "pct_of_measured_hbm": round(100.0 * value / peak, 2),
+        "seq_tokens_per_s": round(tot_tokens / (max_ms * 1e-3), 1),
+        "decode_tokens_per_s": round(tot_seqs / (max_ms * 1e-3), 1),
+        "algorithmic_bytes_per_step": alg_bytes,
+        "logical_bytes_per_step": logical_bytes,
+        "effective_logical_gbs": round(logical_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
+        "gpu_launches": ds.launches_per_step * K,
+        "step_call": "pa_decode_step: " + ("copy_blocks, " if len(step.copy_pairs) else "")
+                     + "plan+scatter prologue, attend, reduce",
+        "step_timing": ("replays of CUDA graphs captured from pa_decode_step calls "
+                        f"({GRAPH_CHUNK} steps per graph back to back, 1 per graph between flushes)"
+                        if graphs is not None else "eager pa_decode_step calls"),
+        "host_enqueue_ms_per_step": round(host_ms / K, 5),
+        "eager": {"ms_per_step": round(eager_ms / K, 5), "host_enqueue_ms_per_step": round(eager_host_ms / K, 5),
+                  "value": round(alg_bytes * K / (eager_ms * 1e-3) / 1e9, 2)},
+        "kv_utilisation": kv_utilisation_summary(step, CONFIGS[name]["max_len"]),
+        "roofline": {
+            "kernel": "attend_bf16_kernel" if step.dtype == torch.bfloat16 else "attend_f32_kernel",
+            "bound": "hbm",
+            "achieved": round(achieved_attend, 2),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+            "unit": "GB/s",
+            "frac": round(achieved_attend / peak, 4),
+            "traffic": traffic,
+            "traffic_source": (f"read from profiles/attend_{name}.ncu.md (an ncu capture of this kernel source, "
+                               "dram__bytes_read.sum + dram__bytes_write.sum per launch), not measured in this run"
+                               if traffic is not None else
+                               "null: no ncu summary of the current attend kernel source for this workload"),
+            "attend_ms": round(attend_ms, 5),
+            "attend_timing": "CUDA events around each attend launch, in a pass after the timed steps "
+                             f"({n_att} launches" + (", L2 flushed before each)" if flush is not None else ")"),
+            "bytes_per_launch": alg_bytes,
+        },
+        "clocks": clock_info,
+        "e2e": e2e_line,
+        "cpu_baseline": cpu,
+        "dtype": "bf16" if step.dtype == torch.bfloat16 else "f32",
+    }
+    del ds, step, flush, graphs
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
-    import numpy as np
     import torch
 
     from paged_kv_cache_382_b200 import build as _build
-    from paged_kv_cache_382_b200 import workloads as W
 
     world, rank, local = dist_setup()
     if world != args.gpus:
@@ -455,143 +697,94 @@ def run_ours(args):
     from paged_kv_cache_382_b200 import pa
 
     dev = torch.device("cuda", local)
-    step = build_step(args.config, args.seed + rank, dev, args.partition_size)
-    ds = DeviceStep(pa, step, args.partition_size)
-    alg_bytes = W.algorithmic_bytes(step, unique=True)
-    logical_bytes = W.algorithmic_bytes(step, unique=False)
-    if ds.prefill:   # q and out hold every new token
-        extra = 2 * (step.q.shape[0] - step.num_seqs) * step.num_heads * step.head_dim * step.element_bytes
-        alg_bytes += extra
-        logical_bytes += extra
-        args.no_e2e = True
-    ctx_tokens = int(step.context_lens.sum())
+    warmup = max(args.warmup, 3)
+    if args.config != DEFAULT_CONFIG and CONFIGS[args.config]["builder"] == "prefill_chunk":
+        run_prefill(args, pa, dev, world, rank, local, pool)
+        return
+    names = ([SUITE_HEADLINE] + [n for n in DECODE_SUITE if n != SUITE_HEADLINE]
+             if args.config == DEFAULT_CONFIG else [args.config])
+    results = {}
+    for i, name in enumerate(names):
+        results[name] = measure_decode(pa, args, name, dev, world, rank, local, args.steps if i == 0 else None,
+                                       warmup, pool if i == 0 else None, cores)
+    if pool is not None:
+        pool.close()
+    if rank != 0:
+        return
+    head = results[names[0]]
+    line = {
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": head["dtype"],
+        "data": "synthetic (seeded; K/V ~ N(0,1) generated on the device by torch, no dataset)",
+        "config": head["config"],
+    }
+    for k in ("pct_of_8tbs", "pct_of_measured_hbm", "seq_tokens_per_s", "decode_tokens_per_s",
+              "algorithmic_bytes_per_step", "logical_bytes_per_step", "effective_logical_gbs", "gpu_launches",
+              "step_call", "step_timing", "host_enqueue_ms_per_step", "eager", "kv_utilisation", "roofline",
+              "clocks", "e2e", "cpu_baseline"):
+        line[k] = head[k]
+    if len(names) > 1:
+        line["per_config"] = {n: {k: v for k, v in r.items() if k not in ("cpu_baseline", "dtype")}
+                              for n, r in results.items()}
+        line["per_config_note"] = (f"every decode workload measured in this run on this GPU; the headline is "
+                                   f"{names[0]} over exactly --steps steps, the others over enough steps to "
+                                   f"fill {PER_CONFIG_MIN_SECONDS} s of device time (at least --steps), stated "
+                                   "per entry")
+    print(json.dumps(line), flush=True)
 
-    stream = torch.cuda.current_stream()
+
+def run_prefill(args, pa, dev, world, rank, local, pool):
+    """The chunked-prefill workload (tensor-core prefill), L2 flushed before every step."""
+    import torch
+
+    from paged_kv_cache_382_b200 import workloads as W
+
+    P = partition_for(args, args.config)
+    step = build_step(args.config, args.seed + rank, dev, P)
+    ds = DeviceStep(pa, step, P)
+    alg_bytes = W.algorithmic_bytes(step, unique=True)
+    alg_bytes += 2 * (step.q.shape[0] - step.num_seqs) * step.num_heads * step.head_dim * step.element_bytes
     for _ in range(max(args.warmup, 3)):
         ds.run()
     torch.cuda.synchronize()
     if int(ds.err.item()) != 0:
         raise RuntimeError(f"device error word {int(ds.err.item()):#x}")
-
     K = args.steps
+    stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     # The chunked-prefill K/V (84 MB) fits the 126 MB L2: flush L2 before every
-    # step (a 256 MB write) and time the steps alone with per-step events.  The
-    # decode workloads' inputs exceed L2 and run back to back.
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if ds.prefill else None
-    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)] if ds.prefill else None
-    # Decode: the timed steps run back to back with nothing between their kernels
-    # (an event between two kernels would cost the programmatic-launch overlap);
-    # the attend kernel alone is timed in a second pass with events around it.
+    # step (a 256 MB write) and time the steps alone with per-step events.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     with ClockSampler(nvsmi_id(local), enabled=not args.no_clocks) as clocks:
         barrier()
         torch.cuda.synchronize()
-        start.record(stream)
         for i in range(K):
-            if flush is not None:
-                flush.fill_(i & 0xFF)
-                ev_step[i][0].record(stream)
-            ds.run(ev_attend=ev[i] if flush is not None else None)
-            if flush is not None:
-                ev_step[i][1].record(stream)
-        stop.record(stream)
+            flush.fill_(i & 0xFF)
+            ev_step[i][0].record(stream)
+            ds.run(ev_attend=ev[i])
+            ev_step[i][1].record(stream)
         torch.cuda.synchronize()
         barrier()
-    elapsed_ms = start.elapsed_time(stop) if flush is None else sum(a.elapsed_time(b) for a, b in ev_step)
-    if flush is None:
-        n_att = min(K, 500)
-        for i in range(n_att):
-            ds.run(ev_attend=ev[i])
-        torch.cuda.synchronize()
-        attend_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev[:n_att])
-    else:
-        attend_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    elapsed_ms = sum(a.elapsed_time(b) for a, b in ev_step)
+    prefill_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
     clock_info = clocks.summary()
-
-    # end to end through the public API: host inputs in, host result out, every step
-    e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(ds, step, alg_bytes, max(args.warmup, 3), min(K, 1000))
-
-    tot_bytes, max_ms, tot_tokens, tot_seqs = reduce_over_ranks(
-        [alg_bytes * K, elapsed_ms, ctx_tokens * K, step.num_seqs * K], ["sum", "max", "sum", "sum"])
-    if e2e is not None:
-        e2e_bytes, e2e_ms = reduce_over_ranks([e2e["bytes"], e2e["ms"]], ["sum", "max"])
-    peak, peak_kind = measured_hbm_peak()
-    achieved_attend = alg_bytes / (attend_ms * 1e-3) / 1e9
-    value = tot_bytes / (max_ms * 1e-3) / 1e9
-
-    cpu = None
+    (max_ms,) = reduce_over_ranks([elapsed_ms], ["max"])
     if pool is not None:
-        if not ds.prefill:
-            cpu = cpu_baseline(step, pool, cores, args.cpu_core_seconds)
         pool.close()
     if rank != 0:
         return
-    if ds.prefill:
-        print(json.dumps(prefill_line(args, step, world, K, max_ms, attend_ms, alg_bytes, clock_info, ds)),
-              flush=True)
-        return
-    traffic = profiled_traffic(args.config)
-    line = {
-        "metric": METRIC,
-        "value": round(value, 2),
-        "unit": UNIT,
-        "n_gpus": world,
-        "steps": K,
-        "warmup": max(args.warmup, 3),
-        "ms_per_step": round(max_ms / K, 5),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16" if step.dtype == torch.bfloat16 else "f32",
-        "data": "synthetic (seeded; K/V ~ N(0,1) generated on the device by torch, no dataset)",
-        "config": {
-            "workload": CONFIGS[args.config]["desc"],
-            "name": args.config,
-            "num_seqs_per_gpu": step.num_seqs,
-            "context_tokens_per_gpu": ctx_tokens,
-            "partition_size": args.partition_size,
-            "parallelism": f"replicas x{world} (independent batches, no collective)",
-            "l2": f"inputs larger than L2: {alg_bytes / 1e9:.3f} GB of K/V+q/out per step vs 126 MB L2",
-        },
-        "pct_of_8tbs": round(100.0 * value / NOMINAL_HBM_GBS, 2),
-        "pct_of_measured_hbm": round(100.0 * value / peak, 2),
-        "seq_tokens_per_s": round(tot_tokens / (max_ms * 1e-3), 1),
-        "decode_tokens_per_s": round(tot_seqs / (max_ms * 1e-3), 1),
-        "algorithmic_bytes_per_step": alg_bytes,
-        "logical_bytes_per_step": logical_bytes,
-        "effective_logical_gbs": round(logical_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
-        "gpu_launches": ds.launches_per_step * K,
-        "step_call": "pa_decode_step: " + ("copy_blocks, " if len(step.copy_pairs) else "")
-                     + "plan+scatter prologue, attend, reduce",
-        "kv_utilisation": kv_utilisation_summary(step, CONFIGS[args.config]["max_len"]),
-        "roofline": {
-            "kernel": "attend_bf16_kernel" if step.dtype == torch.bfloat16 else "attend_f32_kernel",
-            "bound": "hbm",
-            "achieved": round(achieved_attend, 2),
-            "peak": peak,
-            "peak_kind": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                         if peak_kind == "measured" else "fallback 6.65 TB/s",
-            "unit": "GB/s",
-            "frac": round(achieved_attend / peak, 4),
-            "traffic": traffic,
-            "attend_ms": round(attend_ms, 5),
-            "attend_timing": "CUDA events around each attend launch, in a pass after the timed steps "
-                             f"({min(K, 500)} launches)",
-            "bytes_per_launch": alg_bytes,
-        },
-        "clocks": clock_info,
-        "e2e": None,
-        "cpu_baseline": cpu,
-    }
-    if e2e is not None:
-        line["e2e"] = {"value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
-                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "ms_per_step": round(e2e_ms / e2e["steps"], 5), "steps": e2e["steps"]}
-    print(json.dumps(line), flush=True)
+    print(json.dumps(prefill_line(args, step, world, K, max_ms, prefill_ms, alg_bytes, clock_info, ds)),
+          flush=True)
 
 
 def measured_tensor_peak():
@@ -618,7 +811,7 @@ def prefill_line(args, step, world, K, max_ms, prefill_ms, alg_bytes, clock_info
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; K/V/q ~ N(0,1) generated on the device by torch, no dataset)",
         "config": {"workload": CONFIGS[args.config]["desc"], "name": args.config,
-                   "new_tokens_per_gpu": int(step.q.shape[0]), "partition_size": args.partition_size,
+                   "new_tokens_per_gpu": int(step.q.shape[0]), "partition_size": ds.P,
                    "l2": "flushed before every step (256 MB write, outside the per-step CUDA events); "
                          "ms_per_step is the sum of the per-step event times"},
         "kv_gbs": round(alg_bytes * K * world / (max_ms * 1e-3) / 1e9, 2),
@@ -636,13 +829,15 @@ def prefill_line(args, step, world, K, max_ms, prefill_ms, alg_bytes, clock_info
     }
 
 
-def run_e2e(ds, step, alg_bytes, warmup, steps):
+def run_e2e(ds, step, alg_bytes, warmup, steps, flush=None):
     """The same step through the binding, fed from the host: each step's inputs
     (q, new K/V, slot mapping, block tables, context lens) are packed in one
     pinned host buffer and copied in, the step runs, and its output is copied
     back to pinned host memory.  Copies and compute overlap across steps on
     three streams (H2D, compute, D2H) with double-buffered device inputs and
-    outputs, the way a serving loop would feed the kernels."""
+    outputs, the way a serving loop would feed the kernels.  With ``flush`` (a
+    buffer larger than L2) every step instead runs alone after an L2 flush,
+    between its own events: H2D copy, step and D2H copy in series."""
     import torch
 
     parts = dict(q=ds.q, new_key=ds.new_key, new_value=ds.new_value, slots=ds.slots, tables=ds.tables,
@@ -696,6 +891,24 @@ def run_e2e(ds, step, alg_bytes, warmup, steps):
     for i in range(warmup):
         one(i)
     torch.cuda.synchronize()
+    if flush is not None:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            for b in range(2):
+                compute.wait_event(ev_out[b])
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(compute)
+            ev_done[i % 2].record(compute)
+            one(i)
+            compute.wait_event(ev_out[i % 2])
+            ev[i][1].record(compute)
+        torch.cuda.synchronize()
+        barrier()
+        return {"ms": sum(a.elapsed_time(b) for a, b in ev), "bytes": alg_bytes * steps, "h2d": h2d, "d2h": d2h,
+                "steps": steps, "timing": "per step after an L2 flush: H2D copy, step, D2H copy in series, "
+                                          "between events on the compute stream"}
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -709,7 +922,7 @@ def run_e2e(ds, step, alg_bytes, warmup, steps):
     torch.cuda.synchronize()
     barrier()
     return {"ms": start.elapsed_time(stop), "bytes": alg_bytes * steps, "h2d": h2d, "d2h": d2h,
-            "steps": steps}
+            "steps": steps, "timing": "steps pipelined over H2D, compute and D2H streams between two events"}
 
 
 def cpu_baseline(step, pool, cores, core_seconds):
@@ -744,7 +957,9 @@ def run_reference(args):
 
     del W
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))) if torch.cuda.is_available() else "cpu"
-    step = build_step(args.config, args.seed, dev, args.partition_size)
+    name = SUITE_HEADLINE if args.config == DEFAULT_CONFIG else args.config
+    P = partition_for(args, name)
+    step = build_step(name, args.seed, dev, P)
     with tempfile.TemporaryDirectory(prefix="pa_oracle_") as tmp:
         full = OracleSample(step, range(step.num_seqs), pool, tmp)
         wall1, busy1 = full.run(1)
@@ -780,7 +995,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded, same batch as the GPU arm)",
-        "config": {"workload": CONFIGS[args.config]["desc"], "name": args.config},
+        "config": config_dict(name, step, world, P, needs_flush(step)),
         "seq_tokens_per_s": round(total_tokens / total_wall, 1),
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{n_seq} of {len(full.seqs)} sequences per step (every head), "

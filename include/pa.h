@@ -13,8 +13,10 @@
  *    legacy default stream).  Results are ready once the stream reaches the
  *    point of the call.
  *  - Host-side errors (null pointer, bad size, unsupported shape, short
- *    workspace, failed launch) are returned synchronously as a pa_status and
- *    nothing is launched.
+ *    workspace, buffer on another device, failed launch) are returned
+ *    synchronously as a pa_status and nothing is launched.  Right before its
+ *    first launch every call checks that its pool (for pa_selftest_bounded_wait
+ *    the error word) is device memory of the current device.
  *  - Data-dependent errors are found on the device: the offending entry is
  *    skipped (its tokens take no part in the result, the write or copy does
  *    not happen) and a PA_DEVERR_* bit is OR-ed into *dev_err.  dev_err may be
@@ -73,7 +75,10 @@ typedef enum pa_status {
                                  partition_size not a positive multiple of 32 (or > 8192),
                                  dtype combination not offered */
     PA_ERR_WORKSPACE = 3,     /* workspace_bytes below pa_decode_workspace_bytes() */
-    PA_ERR_CUDA = 4           /* a CUDA runtime call or a kernel launch failed */
+    PA_ERR_CUDA = 4,          /* a CUDA runtime call or a kernel launch failed */
+    PA_ERR_DEVICE_INDEX = 5   /* the current CUDA device's index is beyond the library's
+                                 per-device tables (64 devices), or the pool (the call's
+                                 first device buffer) is memory of another device */
 } pa_status;
 
 /* Bits OR-ed into *dev_err by the kernels. */

@@ -67,6 +67,7 @@ extern "C" int pa_selftest_bounded_wait(int32_t* dev_err, uint64_t limit_ns, pa_
     using namespace pa;
     if (!dev_err || !aligned_to(dev_err, 4) || limit_ns == 0 || limit_ns > 1000000000ull)
         return PA_ERR_INVALID_ARG;
+    if (const int rc = device_check(dev_err)) return rc;
     selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns, dev_err);
     return launch_status(cudaGetLastError());
 }
@@ -102,6 +103,7 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
     sa.block_size = block_size;
     sa.num_slots = num_slots;
     sa.dev_err = dev_err;
+    if (const int rc = device_check(k_cache)) return rc;
     return launch_status(launch_pdl(reshape_and_cache_kernel, dim3(num_tokens), dim3(threads), 0,
                                     as_stream(stream), sa));
 }
@@ -123,6 +125,7 @@ extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_d
     if (ctas < 1) ctas = 1;
     if (ctas > 1024) ctas = 1024;
     dim3 grid(static_cast<unsigned>(ctas), static_cast<unsigned>(num_pairs));
+    if (const int rc = device_check(k_cache)) return rc;
     return launch_status(launch_pdl(copy_blocks_kernel, grid, dim3(threads), 0, as_stream(stream),
                                     static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
                                     src_dst_pairs, block_vecs, num_blocks, dev_err));
@@ -135,6 +138,7 @@ extern "C" const char* pa_status_string(int status) {
         case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: shape or dtype not supported";
         case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace too small";
         case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA call or kernel launch failed";
+        case PA_ERR_DEVICE_INDEX: return "PA_ERR_DEVICE_INDEX: device index unsupported or buffer on another device";
         default: return "unknown pa_status";
     }
 }

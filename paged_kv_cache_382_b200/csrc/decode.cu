@@ -14,17 +14,12 @@
 //               sequences whose block tables name the same physical blocks for
 //               a whole partition (parallel samples of one prompt) share one
 //               packed item: one K/V read serves all of them.
-//   2. attend:  persistent CTAs take (item, kv head, head group) units in a
-//               static stride.  One unit = one partition of up to
-//               partition_size tokens of one kv head, for the (up to 8) query
-//               heads that share it, so each K/V byte is read once per group.
-//               bf16: each warp streams 16-token tiles of K and V through its
-//               own ring of shared-memory stages, filled by tensor-map bulk
-//               copies (128-byte swizzle) completing on mbarriers; q.K^T and
-//               p.V run on the tensor cores (m16n8k16, tokens as M, the query
-//               heads as N) with an online softmax in fp32 registers.
-//               fp32: a plain CUDA-core warp-per-token loop.
-//               A sequence that fits one partition writes its output directly;
+//   2. attend:  persistent CTAs take (item, kv head, head group) units, the
+//               first by index, the rest from a ticket.  One unit = one
+//               partition of one kv head for the (up to 32) query columns that
+//               read it (attend_bf16.cuh: tensor-map bulk copies, tensor-core
+//               MMAs, online softmax; fp32: a CUDA-core warp-per-token loop).
+//               A sequence that fits one partition gets its output directly;
 //               otherwise each partition writes (max, sum, unnormalised
 //               output) to the workspace.
 //   3. reduce:  merges the partitions of each multi-partition (seq, head), in a
@@ -42,6 +37,7 @@
 #include <climits>
 #include <cmath>
 
+#include "attend_bf16.cuh"
 #include "pa_device.cuh"
 #include "pa_host.h"
 #include "pa_scatter.cuh"
@@ -68,12 +64,13 @@ struct DecodeArgs {
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks;
     int cap;             // contexts are clamped to [0, cap]
     int partition_size;
+    int log2_block;      // log2(block_size)
     int max_parts;       // ceil(cap / partition_size), at least 1
     int group;           // query heads per kv head
     int head_groups;     // ceil(group / 8): units per kv head
     float scale_log2;    // scale * log2(e)
     int out_f32;         // 1: out is fp32, 0: out is bf16
-    int pack;            // sequences a packed item may serve (8 / group; 1 = no packing)
+    int pack;            // sequences a packed item may serve (32 / group; 1 = no packing)
     const int32_t* row_seq;   // prefill: the sequence (block-table row) of each query row; null = identity
 };
 
@@ -84,13 +81,15 @@ __device__ __forceinline__ const int32_t* table_row(const DecodeArgs& a, int s) 
 }
 
 // A work item names a partition p of sequence s and how many consecutive
-// sequences (s, s+1, ...) share that partition's blocks and are served by it.
+// sequences (s, s+1, ..., at most 32) share that partition's blocks and are
+// served by it.
+constexpr int ITEM_COUNT_BITS = 5;
 __host__ __device__ __forceinline__ int make_item(int s, int p, int count, int max_parts) {
-    return ((s * max_parts + p) << 3) | (count - 1);
+    return ((s * max_parts + p) << ITEM_COUNT_BITS) | (count - 1);
 }
 __device__ __forceinline__ void split_item(int item, int max_parts, int& s, int& p, int& count) {
-    count = (item & 7) + 1;
-    const int sp = item >> 3;
+    count = (item & ((1 << ITEM_COUNT_BITS) - 1)) + 1;
+    const int sp = item >> ITEM_COUNT_BITS;
     s = sp / max_parts;
     p = sp - s * max_parts;
 }
@@ -137,29 +136,44 @@ __device__ int shared_lead(const DecodeArgs& a, int s, int c, int c_next, int fi
 }
 
 // Whole-partition items of sequence s (context c), counted or written to out[].
-// Sequences are packed in aligned runs of a.pack: the first sequence of a run
-// emits one item per partition that its run-mates share with it (consecutive
-// links); a sequence not covered that way emits its own item.  `lead` holds
-// shared_lead of the sequences from lead_base on.
+// Sequences are packed in runs of up to a.pack, aligned at the start of each
+// chain of consecutive sequences that share their first partition (c0 is the
+// start of s's run) and cut at the chunk's end: for each partition, the run's
+// first sequence emits one item for the run-mates linked to it through that
+// partition (consecutive links); a sequence not covered that way emits its
+// own item.  `lead` holds shared_lead of the sequences from lead_base on.
 template <bool WRITE>
-__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int* out) {
+__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int c0, int* out) {
     const int nfull = c / a.partition_size, m = a.pack;
     if (m <= 1) {
         if (WRITE)
             for (int k = 0; k < nfull; ++k) out[k] = make_item(s, k, 1, a.max_parts);
         return nfull;
     }
-    const int c0 = s - s % m, j = s - c0;
+    const int j = s - c0;
+    const int end = min(c0 + m, min(a.num_seqs, lead_base + PLAN_THREADS));
     int n = 0;
     for (int k = 0; k < nfull; ++k) {
         int cnt = 1;
-        while (cnt < m && c0 + cnt < a.num_seqs && lead[c0 + cnt - 1 - lead_base] > k) ++cnt;
+        while (c0 + cnt < end && lead[c0 + cnt - 1 - lead_base] > k) ++cnt;
         if (j == 0 || j >= cnt) {
             if (WRITE) out[n] = make_item(s, k, j == 0 ? cnt : 1, a.max_parts);
             ++n;
         }
     }
     return n;
+}
+
+// Start of s's packing run: runs of a.pack sequences counted from the start of
+// its sharing chain (the first sequence of the chunk, or one that shares no
+// whole partition with its predecessor).  Called by every thread of the CTA.
+__device__ __forceinline__ int run_start(const DecodeArgs& a, int start, const int* lead, int* scratch) {
+    const int t = threadIdx.x;
+    const bool live = start + t < a.num_seqs;
+    const int head = (live && (t == 0 || lead[t - 1] == 0)) ? t : -1;
+    const int chain = cta_inclusive_max_scan(head, scratch);   // -1 identity; t = 0 always starts one
+    if (a.pack <= 1 || !live) return start + t;
+    return start + chain + ((t - chain) / a.pack) * a.pack;
 }
 
 // The plan itself, run by one CTA of PLAN_THREADS threads.
@@ -191,7 +205,8 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
             t = (c % P) != 0 || c == 0;
         }
         __syncthreads();
-        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, nullptr);
+        const int c0 = run_start(a, start, lead, scratch);
+        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, nullptr);
         int cf = 0, ct = 0;
         ef = cta_exclusive_scan(f, &cf, scratch);
         et = cta_exclusive_scan(t, &ct, scratch);
@@ -200,8 +215,9 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
     }
     if (one_chunk) {
         const int s = threadIdx.x;
+        const int c0 = run_start(a, 0, lead, scratch);
         if (s < a.num_seqs) {
-            full_items<true>(a, s, c, lead, 0, a.ws_items + ef);
+            full_items<true>(a, s, c, lead, 0, c0, a.ws_items + ef);
             if (t) a.ws_items[full_total + et] = make_item(s, c / P, 1, a.max_parts);
         }
         if (threadIdx.x == 0) *a.ws_count = full_total + tail_total;
@@ -222,12 +238,13 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
             t = (c % P) != 0 || c == 0;
         }
         __syncthreads();
-        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, nullptr);
+        const int c0 = run_start(a, start, lead, scratch);
+        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, nullptr);
         int chunk_f = 0, chunk_t = 0;
         ef = cta_exclusive_scan(f, &chunk_f, scratch);
         et = cta_exclusive_scan(t, &chunk_t, scratch);
         if (s < a.num_seqs) {
-            full_items<true>(a, s, c, lead, start, a.ws_items + base_full + ef);
+            full_items<true>(a, s, c, lead, start, c0, a.ws_items + base_full + ef);
             if (t) a.ws_items[base_tail + et] = make_item(s, c / P, 1, a.max_parts);
         }
         base_full += chunk_f;
@@ -256,14 +273,14 @@ __global__ void __launch_bounds__(PLAN_THREADS) step_prologue_kernel(const Decod
 }
 
 // ---------------------------------------------------------------------------
-// shared epilogue: merge the W warps' partial softmax states of one unit and
+// fp32 epilogue: merge the W warps' partial softmax states of one unit and
 // store the output row (single partition) or the partition's partial.
 // mm, ml: [W][8] running max (log2 domain) and sum; mo: [W][8][D].
 // ---------------------------------------------------------------------------
 
-// Query row n (0..7, the mma N index) of a unit: the sequence (s + member)
-// and head it belongs to.  Up to 8 / group packed sequences x group heads, or
-// one sequence's heads head0 .. head0+7 when a kv head has more than 8.
+// Query column n of a unit: the sequence (s + member) and head it belongs to.
+// g <= 8: up to 32 / g packed sequences x g heads (n < 32); more heads per kv
+// head: one sequence's heads head0 .. head0+7 (n < 8).
 __device__ __forceinline__ void unit_row(const DecodeArgs& a, int kvh, int hg, int count, int n, int& member,
                                          int& head, bool& valid) {
     if (a.group <= 8) {
@@ -273,7 +290,7 @@ __device__ __forceinline__ void unit_row(const DecodeArgs& a, int kvh, int hg, i
     } else {
         member = 0;
         head = kvh * a.group + hg * 8 + n;
-        valid = n < a.group - hg * 8;
+        valid = n < 8 && n < a.group - hg * 8;
     }
 }
 
@@ -316,48 +333,63 @@ __device__ __forceinline__ void combine_store(const DecodeArgs& a, const float* 
 }
 
 // ---------------------------------------------------------------------------
-// 2a. attend, bf16: tensor-map bulk copies into per-warp stage rings + warp MMA
+// 2a. attend, bf16 (tile arithmetic, stream states and merges: attend_bf16.cuh)
 // ---------------------------------------------------------------------------
 
-// Shared-memory geometry of one 16-token tile.  A K (or V) tile is stored as
-// D/64 "halves" of 64 columns (128 bytes per row) in the 128-byte swizzled
-// layout the bulk copy produces: inside each 1024-byte span, the 16-byte chunk
-// c of row r sits at chunk c ^ (r % 8).  A tile is filled by 16/RB boxes of RB
-// rows (RB = min(block_size, 16)); boxes start on 1024-byte boundaries.
-template <int D, int RB>
-struct TileGeom {
-    static constexpr int NH = D / 64;
-    static constexpr int BOXES = 16 / RB;
-    static constexpr int BOX_STRIDE = RB * 128 >= 1024 ? RB * 128 : 1024;
-    static constexpr int HALF = BOXES * BOX_STRIDE;   // bytes of one 64-column half
-    static constexpr int STAGE = 2 * NH * HALF;       // K halves, then V halves
-    __host__ __device__ static constexpr uint32_t row_off(int r) {
-        return static_cast<uint32_t>((r / RB) * BOX_STRIDE + (r % RB) * 128);
-    }
-};
-
 // Resident CTAs per SM the bf16 attend kernel is register-budgeted for (shared
-// memory allows 4 at 3 warps x 2 stages).
+// memory allows 3 at 4 warps x 2 stages of 8 KB).
 #ifndef PA_ATTEND_MIN_CTAS
-#define PA_ATTEND_MIN_CTAS 4
+#define PA_ATTEND_MIN_CTAS 3
 #endif
+
+// Stores a warp's final state of column group cg (columns 8cg .. 8cg+7) into
+// the epilogue buffers: fin_o[n][D] and fin_ml[n] = (max, sum).
+template <int D>
+__device__ __forceinline__ void store_final(const StreamState<D>& S, float* fin_o, float2* fin_ml, int cg, int g,
+                                            int c) {
+    const int n0 = 8 * cg + 2 * c, n1 = n0 + 1;
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+        fin_o[n0 * D + 16 * i + g] = S.o[i][0];
+        fin_o[n1 * D + 16 * i + g] = S.o[i][1];
+        fin_o[n0 * D + 16 * i + 8 + g] = S.o[i][2];
+        fin_o[n1 * D + 16 * i + 8 + g] = S.o[i][3];
+    }
+    if (g == 0) {
+        fin_ml[n0] = make_float2(S.m0, S.l0);
+        fin_ml[n1] = make_float2(S.m1, S.l1);
+    }
+}
 
 template <int D, int RB, int W, int NS>
 __global__ void __launch_bounds__(W * 32, PA_ATTEND_MIN_CTAS)
 attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const DecodeArgs a) {
     using Geo = TileGeom<D, RB>;
+    using State = StreamState<D>;
     constexpr int NH = Geo::NH, KS = D / 16, HALF = Geo::HALF, STAGE = Geo::STAGE;
-    static_assert(W * NS * STAGE >= W * 8 * (D + 2) * 4, "merge buffers must fit in the stages");
+    constexpr int NSTAGE = W * NS;                               // stage buffers
+    constexpr int SLOT_BYTES = State::FLOATS * 32 * 4;          // one stream state of a warp
+    constexpr int RES = (W * SLOT_BYTES + STAGE - 1) / STAGE;   // stages kept for the merge slots of the
+    constexpr int CS = NSTAGE - RES;                             //   shared layout; the rest form its ring
+    constexpr int FIN = W * SLOT_BYTES;                          // epilogue: final states [32][D], (max, sum) [32]
+    static_assert(W >= 2 && W <= 4, "a unit's columns fill at most W column groups of 8");
+    static_assert(CS >= 2, "the CTA-wide ring needs two stages");
+    static_assert(FIN + 32 * D * 4 + 32 * 8 <= CS * STAGE, "epilogue buffers must sit below the merge slots");
 
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* stages = smem;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + W * NS * STAGE);
-    int* tbl = reinterpret_cast<int*>(bars + W * NS);
+    uint64_t* wbars = reinterpret_cast<uint64_t*>(stages + NSTAGE * STAGE);   // [NSTAGE] per-warp rings
+    uint64_t* cbars = wbars + NSTAGE;                                         // [CS] CTA-wide ring
+    int* ccnt = reinterpret_cast<int*>(cbars + CS);      // [CS] consumers done with the stage's tile
+    int* cissued = ccnt + CS;                            // [CS] tiles ever issued to the stage
+    int* ybase = cissued + CS;   // per block of the partition: tensor-map row of its slot 0, or -1
+    uint16_t* ring_tile = reinterpret_cast<uint16_t*>(ybase + a.partition_size / a.block_size);   // shared layout:
+                                                                      // the tile of each ring position
     __shared__ int s_abort;
-    __shared__ int3 s_rows[8];
+    __shared__ int3 s_rows[32];
     __shared__ unsigned long long s_next;   // the next unit this CTA works on
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -365,10 +397,16 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         s_abort = 0;
         prefetch_tensor_map(&tm_k);
         prefetch_tensor_map(&tm_v);
+#pragma unroll
+        for (int i = 0; i < CS; ++i) {
+            mbar_init(smem_u32(&cbars[i]), 1);
+            ccnt[i] = 0;
+            cissued[i] = 0;
+        }
     }
     if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < NS; ++i) mbar_init(smem_u32(&bars[warp * NS + i]), 1);
+        for (int i = 0; i < NS; ++i) mbar_init(smem_u32(&wbars[warp * NS + i]), 1);
     }
     fence_barrier_init();
     __syncthreads();
@@ -379,24 +417,15 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const long long units = static_cast<long long>(*a.ws_count) * per_item;
     const int P = a.partition_size, B = a.block_size;
     const float sl2 = a.scale_log2;
-
-    // Fragment coordinates of this lane.
-    const int g = lane >> 2, c = lane & 3;         // mma C/B fragment row group and column pair
-    const int mi = lane >> 3, rr = lane & 7;       // ldmatrix: matrix index and row within it
-    const uint32_t krow = Geo::row_off(rr + 8 * (mi & 1));
-    const uint32_t vrow = Geo::row_off(rr + 8 * (mi >> 1));
-    const uint32_t ksw = (krow >> 7) & 7, vsw = (vrow >> 7) & 7;
-    uint32_t kx[4], vx[4];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-        kx[q4] = ((2 * q4 + (mi >> 1)) ^ ksw) << 4;
-        vx[q4] = ((2 * q4 + (mi & 1)) ^ vsw) << 4;
-    }
-
-    uint8_t* wst = stages + warp * NS * STAGE;
-    const uint32_t wst_u32 = smem_u32(wst);
-    const uint32_t wbar_u32 = smem_u32(&bars[warp * NS]);
+    const int g = lane >> 2, c = lane & 3;   // mma C/B fragment row group and column pair
+    const LaneFrag<D, RB> frag(lane);
+    const uint32_t stages_u32 = smem_u32(stages);
+    const uint32_t wst_u32 = stages_u32 + warp * NS * STAGE;
+    const uint32_t wbar_u32 = smem_u32(&wbars[warp * NS]);
     uint32_t n_issued = 0, n_used = 0;   // this warp's ring position; carried across units
+    uint32_t ring_base = 0;              // tiles passed through the CTA-wide ring (same in every thread)
+    float* fin_o = reinterpret_cast<float*>(stages + FIN);
+    float2* fin_ml = reinterpret_cast<float2*>(stages + FIN + 32 * D * 4);
 
     // CTA b starts with unit b; later units come from a ticket in plan order
     // (whole partitions first), so a CTA that drew short units takes more.
@@ -418,6 +447,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int ntok = t1 - t0;
         const int nblk = ntok > 0 ? (t1 - 1) / B - t0 / B + 1 : 0;
         const int nrows = unit_rows(a, hg, count);
+        const int ncg = (nrows + 7) / 8;   // column groups: > 1 only for packed items (whole partitions)
 
         __syncthreads();   // the previous unit's epilogue is done with shared memory; s_next read
         if (s_abort) break;
@@ -428,7 +458,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             if (v + 1 == static_cast<unsigned long long>(units)) *a.ws_ticket = 0ull;
             s_next = gridDim.x + v;
         }
-        if (tid < 8) {
+        if (tid < 32) {
             int member, head;
             bool valid;
             unit_row(a, kvh, hg, count, tid, member, head, valid);
@@ -436,212 +466,291 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             s_rows[tid] = make_int3(s + member, head, (cm + P - 1) / P);
         }
 
-        // block-table slice of this partition, validated once
+        // block-table slice of this partition, validated once and turned into
+        // the tensor-map row of each block's first slot for this kv head
         int bad = 0;
         const int32_t* trow = table_row(a, s) + t0 / B;
         for (int i = tid; i < nblk; i += W * 32) {
-            int b = trow[i];
-            if (b < 0 || b >= a.num_blocks) {
-                b = -1;
+            const int b = trow[i];
+            int y = -1;
+            if (b < 0 || b >= a.num_blocks)
                 bad = 1;
-            }
-            tbl[i] = b;
+            else
+                y = (b * a.num_kv_heads + kvh) * B;
+            ybase[i] = y;
         }
-        // q fragments (B operand of S^T = K Q^T): query row g, columns 16ks + 2c (+8)
-        uint32_t qf[KS][2];
-        int q_member, q_head;
-        bool q_valid;
-        unit_row(a, kvh, hg, count, g, q_member, q_head, q_valid);
-        if (q_valid) {
-            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-                static_cast<const __nv_bfloat16*>(a.q) +
-                (static_cast<size_t>(s + q_member) * a.num_heads + q_head) * D);
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                qf[ks][0] = qrow[8 * ks + c];
-                qf[ks][1] = qrow[8 * ks + c + 4];
+        const int ntiles = (ntok + 15) / 16;
+        const int qn = ntiles / W, rem = ntiles - qn * W;   // streams 0..rem-1 hold qn + 1 tiles
+        if (ncg > 1) {
+            // the CTA ring passes the tiles in stream order: stream 0's, then stream 1's, ...
+            for (int j = tid; j < ntiles; j += W * 32) {
+                const int sj = j % W, tj = j / W;
+                ring_tile[sj * qn + min(sj, rem) + tj] = static_cast<uint16_t>(j);
             }
-        } else {
+        }
+        // q fragments (B operand of S^T = K Q^T) of the lane's column g of its
+        // warp's column group: d = 16ks + 2c (+8)
+        const int cg = ncg > 1 ? warp : 0;
+        uint32_t qf[KS][2];
+        {
+            int q_member, q_head;
+            bool q_valid;
+            unit_row(a, kvh, hg, count, 8 * cg + g, q_member, q_head, q_valid);
+            if (q_valid && cg < ncg) {
+                const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                    static_cast<const __nv_bfloat16*>(a.q) +
+                    (static_cast<size_t>(s + q_member) * a.num_heads + q_head) * D);
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) qf[ks][0] = qf[ks][1] = 0u;
+                for (int ks = 0; ks < KS; ++ks) {
+                    qf[ks][0] = qrow[8 * ks + c];
+                    qf[ks][1] = qrow[8 * ks + c + 4];
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) qf[ks][0] = qf[ks][1] = 0u;
+            }
         }
         bad = __syncthreads_or(bad);
         if (bad && tid == 0) flag_error(a.dev_err, PA_DEVERR_BLOCK_ID);
+        const int lb = a.log2_block;
 
-        const int ntiles = (ntok + 15) / 16;
-        const int my_tiles = warp < ntiles ? (ntiles - warp + W - 1) / W : 0;
+        State S;
+        S.reset();
+        bool failed = false;
 
-        // Issue the bulk copies of this warp's j-th tile into the next ring stage.
-        auto issue = [&](int j) {
-            const int stage = static_cast<int>(n_issued % NS);
-            ++n_issued;
-            if (lane == 0) {
+        if (ncg == 1) {
+            // ---- one column group: warp w runs stream w through its own ring
+            const int my_tiles = warp < ntiles ? (ntiles - warp + W - 1) / W : 0;   // = qn + (warp < rem)
+            // Issue the bulk copies of this warp's j-th tile into the next ring stage.
+            auto issue = [&](int j) {
+                const int stage = static_cast<int>(n_issued % NS);
+                ++n_issued;
+                if (lane == 0) {
+                    const int r0 = 16 * (warp + j * W);
+                    const uint32_t bar = wbar_u32 + 8 * stage;
+                    const uint32_t dst = wst_u32 + stage * STAGE;
+                    int y[Geo::BOXES];
+                    uint32_t bytes = 0;
+#pragma unroll
+                    for (int piece = 0; piece < Geo::BOXES; ++piece) {
+                        const int tok = r0 + piece * RB;
+                        y[piece] = tok < ntok ? ybase[tok >> lb] : -1;
+                        if (y[piece] >= 0) {
+                            y[piece] += tok & (B - 1);
+                            bytes += 2 * NH * RB * 128;
+                        }
+                    }
+                    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+                    for (int piece = 0; piece < Geo::BOXES; ++piece) {
+                        if (y[piece] < 0) continue;
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) {
+                            tma_load_2d(dst + h * HALF + piece * Geo::BOX_STRIDE, &tm_k, bar, 64 * h, y[piece]);
+                            tma_load_2d(dst + (NH + h) * HALF + piece * Geo::BOX_STRIDE, &tm_v, bar, 64 * h,
+                                        y[piece]);
+                        }
+                    }
+                }
+            };
+            const int npro = my_tiles < NS ? my_tiles : NS;
+            for (int j = 0; j < npro; ++j) issue(j);
+            for (int j = 0; j < my_tiles; ++j) {
+                const int stage = static_cast<int>(n_used % NS);
+                const uint32_t parity = (n_used / NS) & 1u;
+                const bool arrived = mbar_wait_bounded(wbar_u32 + 8 * stage, parity, WAIT_LIMIT_NS);
+                if (!__all_sync(FULL_MASK, arrived)) {   // keep the warp together on a timeout
+                    failed = true;
+                    break;
+                }
+                ++n_used;
+                const uint32_t st = wst_u32 + stage * STAGE;
                 const int r0 = 16 * (warp + j * W);
-                const uint32_t bar = wbar_u32 + 8 * stage;
-                const uint32_t dst = wst_u32 + stage * STAGE;
+                // tokens of this tile that take part: inside the partition and in a valid block
+                unsigned mask = 0xffffu;
+                if (r0 + 16 > ntok || bad) {
+                    const int tok = r0 + (lane & 15);
+                    const bool ok = tok < ntok && ybase[tok >> lb] >= 0;
+                    mask = __ballot_sync(FULL_MASK, ok) & 0xffffu;
+                    // value rows of excluded tokens may hold anything (NaN included): zero them
+                    uint8_t* stp = stages + warp * NS * STAGE + stage * STAGE;
+                    for (int idx = lane; idx < 16 * NH * 8; idx += 32) {
+                        const int row = idx / (NH * 8), rem = idx % (NH * 8);
+                        if (!((mask >> row) & 1u))
+                            *reinterpret_cast<uint4*>(stp + (NH + rem / 8) * HALF + Geo::row_off(row) +
+                                                      (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                attend_tile<D, RB>(S, st, qf, mask, sl2, frag, g);
+                __syncwarp();
+                if (j + NS < my_tiles) issue(j + NS);
+            }
+            if (failed) {
+                // wait, again bounded, for this warp's copies still in flight
+                while (n_used < n_issued) {
+                    const int stage = static_cast<int>(n_used % NS);
+                    mbar_wait_bounded(wbar_u32 + 8 * stage, (n_used / NS) & 1u, DRAIN_LIMIT_NS);
+                    ++n_used;
+                }
+            }
+            S.reduce_sums();
+        } else {
+            // ---- several column groups (a whole partition shared by several
+            // sequences): warp cg runs every stream of column group cg, and each
+            // tile passes once through the CTA-wide ring, in stream order
+            // (stream 0's tiles, then stream 1's, ...), read by all ncg warps.
+            // The last warp done with a stage refills it.
+            auto issue_cta = [&](int k) {   // ring position k of this unit
+                const int r0 = 16 * static_cast<int>(ring_tile[k]);
+                const int stage = static_cast<int>((ring_base + k) % CS);
+                const uint32_t bar = smem_u32(&cbars[stage]);
+                const uint32_t dst = stages_u32 + stage * STAGE;
+                int y[Geo::BOXES];
                 uint32_t bytes = 0;
+                bool zeroed = false;
 #pragma unroll
                 for (int piece = 0; piece < Geo::BOXES; ++piece) {
-                    const int tok = r0 + piece * RB;
-                    if (tok < ntok && tbl[tok / B] >= 0) bytes += 2 * NH * RB * 128;
+                    const int tok = r0 + piece * RB;   // whole partitions: every tile is full
+                    y[piece] = ybase[tok >> lb];
+                    if (y[piece] >= 0) {
+                        y[piece] += tok & (B - 1);
+                        bytes += 2 * NH * RB * 128;
+                    } else {
+                        // a block the table cannot name: its value rows become zero
+                        // (its logits are masked by every reader)
+                        uint8_t* stp = stages + stage * STAGE;
+                        for (int idx = 0; idx < RB * NH * 8; ++idx) {
+                            const int row = piece * RB + idx / (NH * 8), q16 = idx % (NH * 8);
+                            *reinterpret_cast<uint4*>(stp + (NH + q16 / 8) * HALF + Geo::row_off(row) +
+                                                      (q16 % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        zeroed = true;
+                    }
                 }
+                if (zeroed) fence_proxy_async_smem();
+                ++cissued[stage];
                 mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
                 for (int piece = 0; piece < Geo::BOXES; ++piece) {
-                    const int tok = r0 + piece * RB;
-                    if (tok >= ntok) break;
-                    const int phys = tbl[tok / B];
-                    if (phys < 0) continue;
-                    const int y = (phys * a.num_kv_heads + kvh) * B + (tok % B);
+                    if (y[piece] < 0) continue;
 #pragma unroll
                     for (int h = 0; h < NH; ++h) {
-                        tma_load_2d(dst + h * HALF + piece * Geo::BOX_STRIDE, &tm_k, bar, 64 * h, y);
-                        tma_load_2d(dst + (NH + h) * HALF + piece * Geo::BOX_STRIDE, &tm_v, bar, 64 * h, y);
+                        tma_load_2d(dst + h * HALF + piece * Geo::BOX_STRIDE, &tm_k, bar, 64 * h, y[piece]);
+                        tma_load_2d(dst + (NH + h) * HALF + piece * Geo::BOX_STRIDE, &tm_v, bar, 64 * h, y[piece]);
                     }
                 }
+            };
+            if (tid == 0) {
+                const int npro = ntiles < CS ? ntiles : CS;
+                for (int k = 0; k < npro; ++k) issue_cta(k);
             }
-        };
-
-        float m0 = NEG_INF, m1 = NEG_INF, l0 = 0.f, l1 = 0.f;
-        float o[KS][4];
-#pragma unroll
-        for (int i = 0; i < KS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-
-        const int npro = my_tiles < NS ? my_tiles : NS;
-        for (int j = 0; j < npro; ++j) issue(j);
-
-        bool failed = false;
-        for (int j = 0; j < my_tiles; ++j) {
-            const int stage = static_cast<int>(n_used % NS);
-            const uint32_t parity = (n_used / NS) & 1u;
-            const bool arrived = mbar_wait_bounded(wbar_u32 + 8 * stage, parity, WAIT_LIMIT_NS);
-            if (!__all_sync(FULL_MASK, arrived)) {   // keep the warp together on a timeout
-                failed = true;
-                break;
-            }
-            ++n_used;
-            const uint32_t st = wst_u32 + stage * STAGE;
-            const int r0 = 16 * (warp + j * W);
-
-            // tokens of this tile that take part: inside the partition and in a valid block
-            unsigned mask = 0xffffu;
-            if (r0 + 16 > ntok || bad) {
-                const int tok = r0 + (lane & 15);
-                const bool ok = tok < ntok && tbl[tok / B] >= 0;
-                mask = __ballot_sync(FULL_MASK, ok) & 0xffffu;
-                // value rows of excluded tokens may hold anything (NaN included): zero them
-                uint8_t* stp = wst + stage * STAGE;
-                for (int idx = lane; idx < 16 * NH * 8; idx += 32) {
-                    const int row = idx / (NH * 8), rem = idx % (NH * 8);
-                    if (!((mask >> row) & 1u))
-                        *reinterpret_cast<uint4*>(stp + (NH + rem / 8) * HALF + Geo::row_off(row) +
-                                                  (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-
-            // S^T (16 tokens x 8 heads) = K (16 x D) . Q^T (D x 8), as two independent
-            // accumulation chains (even / odd k-steps) to halve the MMA dependency chain
-            float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < KS; ks += 2) {
-                uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
-                ldmatrix_x4(st + (ks / 4) * HALF + krow + kx[ks % 4], a0, a1, a2, a3);
-                ldmatrix_x4(st + ((ks + 1) / 4) * HALF + krow + kx[(ks + 1) % 4], e0, e1, e2, e3);
-                mma_bf16_16816(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-                mma_bf16_16816(sd, e0, e1, e2, e3, qf[ks + 1][0], qf[ks + 1][1]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) sc[i] += sd[i];
-            // logits in the log2 domain; rows g and g+8 are tokens, columns 2c, 2c+1 heads
-            float x0 = sc[0] * sl2, x1 = sc[1] * sl2, x2 = sc[2] * sl2, x3 = sc[3] * sl2;
-            if (mask != 0xffffu) {
-                if (!((mask >> g) & 1u)) x0 = x1 = NEG_INF;
-                if (!((mask >> (g + 8)) & 1u)) x2 = x3 = NEG_INF;
-            }
-            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
-            }
-            const bool up0 = mx0 > m0 + RESCALE_THRESHOLD, up1 = mx1 > m1 + RESCALE_THRESHOLD;
-            if (__any_sync(FULL_MASK, up0 || up1)) {
-                const float al0 = up0 ? exp2_approx(m0 - mx0) : 1.f;
-                const float al1 = up1 ? exp2_approx(m1 - mx1) : 1.f;
-                if (up0) m0 = mx0;
-                if (up1) m1 = mx1;
-                l0 *= al0;
-                l1 *= al1;
-#pragma unroll
-                for (int i = 0; i < KS; ++i) {
-                    o[i][0] *= al0;
-                    o[i][1] *= al1;
-                    o[i][2] *= al0;
-                    o[i][3] *= al1;
+            if (warp < ncg) {
+                float* aslot = reinterpret_cast<float*>(stages + CS * STAGE + warp * SLOT_BYTES);
+                int k = 0;
+                for (int sidx = 0; sidx < W; ++sidx) {
+                    if (sidx > 0) S.reset();
+                    const int cnt = sidx < rem ? qn + 1 : qn;
+                    for (int t = 0; t < cnt; ++t, ++k) {
+                        const uint32_t pos = ring_base + static_cast<uint32_t>(k);
+                        const int stage = static_cast<int>(pos % CS);
+                        const bool arrived =
+                            mbar_wait_bounded(smem_u32(&cbars[stage]), (pos / CS) & 1u, WAIT_LIMIT_NS);
+                        if (!__all_sync(FULL_MASK, arrived)) {
+                            failed = true;
+                            break;
+                        }
+                        unsigned mask = 0xffffu;
+                        if (bad) {
+                            const int tok = 16 * (sidx + W * t) + (lane & 15);
+                            mask = __ballot_sync(FULL_MASK, ybase[tok >> lb] >= 0) & 0xffffu;
+                        }
+                        attend_tile<D, RB>(S, stages_u32 + stage * STAGE, qf, mask, sl2, frag, g);
+                        __syncwarp();
+                        // this warp is done with the stage (its reads ordered before the
+                        // count); the last of the ncg readers refills it
+                        if (lane == 0 && atomic_add_acq_rel_cta(&ccnt[stage], 1) == ncg - 1) {
+                            ccnt[stage] = 0;
+                            if (k + CS < ntiles) issue_cta(k + CS);
+                        }
+                    }
+                    if (failed) break;
+                    S.reduce_sums();
+                    // streams merge in order: slot = s0, then slot (+) s1, (+) s2; the
+                    // last stream's merge leaves the column group's final state in S
+                    if (sidx == 0)
+                        S.store(aslot, lane);
+                    else if (sidx < W - 1)
+                        merge_into_slot<D>(aslot, S, lane);
+                    else
+                        merge_slot_first<D>(S, aslot, lane);
                 }
             }
-            const float b0 = m0 == NEG_INF ? 0.f : m0, b1 = m1 == NEG_INF ? 0.f : m1;
-            const float p0 = exp2_approx(x0 - b0), p1 = exp2_approx(x1 - b1);
-            const float p2 = exp2_approx(x2 - b0), p3 = exp2_approx(x3 - b1);
-            l0 += p0 + p2;
-            l1 += p1 + p3;
-            // weights as a bf16 pair hi + lo (about 16 significant bits), transposed
-            // into the B operand of O^T (D x 8) += V^T (D x 16) . P^T (16 x 8)
-            const uint32_t h01 = pack_bf16(p0, p1), h23 = pack_bf16(p2, p3);
-            const uint32_t q01 = pack_bf16(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
-            const uint32_t q23 = pack_bf16(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
-            const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
-            const uint32_t bl0 = movmatrix_trans(q01), bl1 = movmatrix_trans(q23);
-#pragma unroll
-            for (int i = 0; i < KS; ++i) {
-                uint32_t a0, a1, a2, a3;
-                ldmatrix_x4_trans(st + (NH + i / 4) * HALF + vrow + vx[i % 4], a0, a1, a2, a3);
-                mma_bf16_16816(o[i], a0, a1, a2, a3, bh0, bh1);
-                mma_bf16_16816(o[i], a0, a1, a2, a3, bl0, bl1);
-            }
-            __syncwarp();
-            if (j + NS < my_tiles) issue(j + NS);
+            ring_base += static_cast<uint32_t>(ntiles);
         }
-        if (failed) {
-            if (lane == 0) {
+
+        if (__syncthreads_or(failed)) {   // every warp is done with the stages either way
+            if (tid == 0) {
                 flag_error(a.dev_err, PA_DEVERR_TIMEOUT);
                 s_abort = 1;
+                if (ncg > 1) {   // wait, again bounded, for the CTA ring's copies still in flight
+                    for (int st = 0; st < CS; ++st)
+                        if (cissued[st] > 0)
+                            mbar_wait_bounded(smem_u32(&cbars[st]), (cissued[st] - 1) & 1, DRAIN_LIMIT_NS);
+                }
             }
-            // wait, again bounded, for this warp's copies still in flight
-            while (n_used < n_issued) {
-                const int stage = static_cast<int>(n_used % NS);
-                mbar_wait_bounded(wbar_u32 + 8 * stage, (n_used / NS) & 1u, DRAIN_LIMIT_NS);
-                ++n_used;
-            }
+            break;
         }
-
-        // row sums over the 8 lanes that share a head pair
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l0 += __shfl_xor_sync(FULL_MASK, l0, off);
-            l1 += __shfl_xor_sync(FULL_MASK, l1, off);
-        }
-        __syncthreads();   // every warp is done with its stages
-        float* mm = reinterpret_cast<float*>(stages);
-        float* ml = mm + W * 8;
-        float* mo = ml + W * 8;
-        if (g == 0) {
-            mm[warp * 8 + 2 * c] = m0;
-            mm[warp * 8 + 2 * c + 1] = m1;
-            ml[warp * 8 + 2 * c] = l0;
-            ml[warp * 8 + 2 * c + 1] = l1;
-        }
-#pragma unroll
-        for (int i = 0; i < KS; ++i) {
-            mo[(warp * 8 + 2 * c) * D + 16 * i + g] = o[i][0];
-            mo[(warp * 8 + 2 * c + 1) * D + 16 * i + g] = o[i][1];
-            mo[(warp * 8 + 2 * c) * D + 16 * i + 8 + g] = o[i][2];
-            mo[(warp * 8 + 2 * c + 1) * D + 16 * i + 8 + g] = o[i][3];
+        const float* slots = reinterpret_cast<const float*>(stages);
+        if (ncg == 1) {
+            // the W stream states wait in slots; every thread merges some of the
+            // unit's (column, element) pairs, streams in order (the arithmetic of
+            // merge_into_slot / merge_slot_first, element by element)
+            S.store(reinterpret_cast<float*>(stages + warp * SLOT_BYTES), lane);
+        } else if (warp < ncg) {
+            store_final<D>(S, fin_o, fin_ml, warp, g, c);
         }
         __syncthreads();
-        combine_store<W, D>(a, mm, ml, mo, s_rows, p, nrows);
+        for (int idx = tid; idx < nrows * D; idx += W * 32) {
+            const int n = idx / D, d = idx - (idx / D) * D;
+            const int3 ri = s_rows[n];
+            float O;
+            float2 ml;
+            if (ncg == 1) {
+                // lane (g, c) holds columns 2c, 2c+1 and elements 16i + g (+8)
+                const int e = (n & 1) + 2 * ((d >> 3) & 1), i16 = d >> 4;
+                const int ol = 4 * (d & 7) + (n >> 1), sl = n >> 1;    // lane holding (n, d); a lane of column n
+                const int km = n & 1, ko = 4 + 4 * i16 + e;
+                float M = slots[km * 32 + sl], L = slots[(2 + km) * 32 + sl];
+                O = slots[ko * 32 + ol];
+#pragma unroll
+                for (int w = 1; w < W; ++w) {
+                    const float* sw = slots + w * (SLOT_BYTES / 4);
+                    float Mn, ca, cb;
+                    merge_coef(M, sw[km * 32 + sl], Mn, ca, cb);
+                    L = merge_val(ca, L, cb, sw[(2 + km) * 32 + sl]);
+                    O = merge_val(ca, O, cb, sw[ko * 32 + ol]);
+                    M = Mn;
+                }
+                ml = make_float2(M, L);
+            } else {
+                O = fin_o[idx];
+                ml = fin_ml[n];
+            }
+            const size_t row = static_cast<size_t>(ri.x) * a.num_heads + ri.y;
+            if (ri.z <= 1) {
+                const float v = ml.y > 0.f ? O / ml.y : 0.f;
+                if (a.out_f32)
+                    static_cast<float*>(a.out)[row * D + d] = v;
+                else
+                    static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(v);
+            } else {
+                const size_t slot = row * a.max_parts + p;
+                a.ws_acc[slot * D + d] = O;
+                if (d == 0) a.ws_ml[slot] = ml;
+            }
+        }
         fence_proxy_async_smem();   // these generic accesses precede the next unit's bulk copies
     }
 }
@@ -917,7 +1026,7 @@ prefill_rows_kernel(const int32_t* __restrict__ context_lens, const int32_t* __r
 // ---------------------------------------------------------------------------
 
 #ifndef PA_ATTEND_WARPS
-#define PA_ATTEND_WARPS 3
+#define PA_ATTEND_WARPS 4
 #endif
 #ifndef PA_ATTEND_STAGES
 #define PA_ATTEND_STAGES 2
@@ -963,7 +1072,10 @@ int launch_attend_bf16(const DecodeArgs& a, cudaStream_t st, long long unit_boun
         !encode_pool_map(&tv, a.v_cache, a.num_blocks, a.num_kv_heads, a.block_size, D, RB))
         return PA_ERR_CUDA;
     const int tbl_entries = a.partition_size / a.block_size;
-    const int smem = 1024 + W * NS * Geo::STAGE + W * NS * 8 + tbl_entries * 4;
+    // stages, per-warp and CTA-ring barriers (<= W * NS each), the ring's two
+    // counters per stage, the table slice
+    const int smem = 1024 + W * NS * Geo::STAGE + 2 * W * NS * 8 + 2 * W * NS * 4 + tbl_entries * 4 +
+                     (a.partition_size / 16) * 2;
     auto kern = attend_bf16_kernel<D, RB, W, NS>;
     const int per_sm = prepare_kernel(slot, reinterpret_cast<const void*>(kern), W * 32, smem);
     int dev = 0;
@@ -1050,7 +1162,7 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
 
     const long long cap = context_cap(max_blocks_per_seq, block_size, max_context_len);
     const int max_parts = parts_for(static_cast<int>(cap), partition_size);
-    if (static_cast<long long>(num_seqs) * max_parts > INT_MAX / 16) return PA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(num_seqs) * max_parts > (INT_MAX >> ITEM_COUNT_BITS)) return PA_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, max_parts);
     if (!workspace || !aligned_to(workspace, 256)) return PA_ERR_INVALID_ARG;
     if (workspace_bytes < L.total) return PA_ERR_WORKSPACE;
@@ -1088,16 +1200,19 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
     a.max_blocks = max_blocks_per_seq;
     a.cap = static_cast<int>(cap);
     a.partition_size = partition_size;
+    a.log2_block = block_size == 4 ? 2 : block_size == 8 ? 3 : block_size == 16 ? 4 : 5;
     a.max_parts = max_parts;
     a.group = num_heads / num_kv_heads;
     a.head_groups = (a.group + 7) / 8;
     a.scale_log2 = scale * LOG2E;
     a.out_f32 = out_dtype == PA_F32;
     a.row_seq = row_seq;
-    // bf16 units hold 8 query columns: up to 8 / group sequences sharing a
-    // partition's blocks can share one unit (fp32 units are never packed)
-    a.pack = (dtype == PA_BF16 && a.group <= 4) ? 8 / a.group : 1;
+    // bf16 units hold up to 8 query columns per warp: up to 8 * ATTEND_WARPS /
+    // group sequences sharing a partition's blocks share one unit (fp32 units
+    // are never packed)
+    a.pack = (dtype == PA_BF16 && a.group <= 8) ? 8 * ATTEND_WARPS / a.group : 1;
     const cudaStream_t st = as_stream(stream);
+    if (const int rc = device_check((phases & PA_PHASE_ATTEND) ? k_cache : context_lens)) return rc;
 
     if (prep(st, a.cap) != PA_OK) return PA_ERR_CUDA;
     if (phases & PA_PHASE_PLAN) {
@@ -1203,6 +1318,7 @@ extern "C" int pa_prefill(void* out, pa_dtype out_dtype, const void* q, const vo
             !aligned_to(v_cache, 16) || !aligned_to(block_tables, 4))
             return PA_ERR_INVALID_ARG;
         const long long cap = context_cap(max_blocks_per_seq, block_size, max_context_len);
+        if (const int drc = device_check(k_cache)) return drc;
         return prefill_tc(out, out_dtype, q, k_cache, v_cache, block_tables, context_lens, query_start, num_seqs,
                           num_tokens, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
                           max_blocks_per_seq, static_cast<int>(cap), scale, workspace, workspace_bytes, dev_err,

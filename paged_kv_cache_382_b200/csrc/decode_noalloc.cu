@@ -55,16 +55,10 @@ extern "C" int pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* q, c
                                  int max_blocks_per_seq, int max_context_len, float scale,
                                  int partition_size, pa_dtype dtype, int32_t* dev_err,
                                  pa_stream stream) {
-    // The same context bound pa_decode uses, so the size check matches its needs.
-    if (max_blocks_per_seq > 0 && block_size > 0 && max_context_len >= 0) {
-        long long cap = static_cast<long long>(max_blocks_per_seq) * block_size;
-        if (max_context_len > 0 && max_context_len < cap) cap = max_context_len;
-        if (cap <= 2147483647LL) {
-            const size_t need = pa_decode_workspace_bytes(num_seqs, num_heads, head_dim,
-                                                          static_cast<int>(cap), partition_size);
-            if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
-        }
-    }
+    // The array is handed to pa_decode's own code as a workspace of
+    // PA_NOALLOC_SCRATCH_BYTES: the shapes are checked first, then a batch
+    // needing more than the array gets PA_ERR_WORKSPACE, with nothing launched,
+    // exactly as pa_decode answers a short caller workspace.
     void* scratch = scratch_on_current_device();
     if (scratch == nullptr) return PA_ERR_CUDA;
     return pa_decode_phases(out, out_dtype, q, k_cache, v_cache, block_tables, context_lens, num_seqs,

@@ -139,6 +139,18 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Atomic add on shared memory with acquire-release semantics at CTA scope: this
+// thread's earlier memory accesses are ordered before it, and accesses that
+// preceded the other threads' adds it observes are ordered before its later ones.
+__device__ __forceinline__ int atomic_add_acq_rel_cta(int* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "r"(smem_u32(p)), "r"(v)
+                 : "memory");
+    return old;
+}
+
 // ---- block-wide prefix sums --------------------------------------------------
 
 __device__ __forceinline__ int warp_inclusive_scan(int v) {
@@ -168,6 +180,33 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* total, int* scratc
     __syncthreads();
     *total = scratch[32];
     return scratch[warp] + inc - v;
+}
+
+__device__ __forceinline__ int warp_inclusive_max_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(FULL_MASK, v, o);
+        if (lane >= o) v = max(v, n);
+    }
+    return v;
+}
+
+// Inclusive prefix maximum of v (values >= -1; -1 is the identity) over the
+// CTA.  `scratch` holds 33 ints.
+__device__ __forceinline__ int cta_inclusive_max_scan(int v, int* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int inc = warp_inclusive_max_scan(v);
+    __syncthreads();
+    if (lane == 31) scratch[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int x = lane < nw ? scratch[lane] : -1;
+        const int xi = warp_inclusive_max_scan(x);
+        if (lane < nw) scratch[lane] = xi;
+    }
+    __syncthreads();
+    return warp > 0 ? max(scratch[warp - 1], inc) : inc;
 }
 
 // ---- numerics ----------------------------------------------------------------

@@ -26,6 +26,29 @@ inline bool valid_dtype(int dt) { return dt == PA_F32 || dt == PA_BF16; }
 
 constexpr int MAX_DEVICES = 64;
 
+// Checks, right before a launch, that the current device can be served and that
+// `buf` (a buffer the launch reads or writes; may be null) lives on it:
+// PA_ERR_DEVICE_INDEX if the device index is beyond the per-device tables or
+// `buf` is device memory of another GPU, PA_ERR_INVALID_ARG if `buf` is host
+// memory the GPU cannot reach, PA_ERR_CUDA if the runtime cannot be queried.
+inline int device_check(const void* buf) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return PA_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= MAX_DEVICES) return PA_ERR_DEVICE_INDEX;
+    if (buf == nullptr) return PA_OK;
+    cudaPointerAttributes at = {};
+    if (cudaPointerGetAttributes(&at, buf) != cudaSuccess) {
+        cudaGetLastError();
+        return PA_ERR_INVALID_ARG;
+    }
+    if (at.type == cudaMemoryTypeUnregistered) return PA_ERR_INVALID_ARG;
+    if (at.type == cudaMemoryTypeDevice && at.device != dev) return PA_ERR_DEVICE_INDEX;
+    return PA_OK;
+}
+
 // Number of SMs of the current device (queried once per device).
 inline int current_sm_count(int* device_out = nullptr) {
     static std::atomic<int> cache[MAX_DEVICES];

@@ -19,7 +19,7 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
 
 PA_F32, PA_BF16 = 0, 1
-PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, 1, 2, 3, 4
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_DEVICE_INDEX = 0, 1, 2, 3, 4, 5
 DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_CONTEXT, DEVERR_COPY, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
 PHASE_PLAN, PHASE_ATTEND, PHASE_REDUCE, PHASE_ALL = 0x1, 0x2, 0x4, 0x7
 

@@ -80,7 +80,10 @@ class DecodeStep:
 
 
 def algorithmic_bytes(step: DecodeStep, unique: bool = True) -> int:
-    """Bytes the decode of one layer must move, by the model stated in DESIGN:
+    """Bytes the decode of one layer must move: every valid token's K and V
+    gathered once through the block table ("PagedAttention blog" section 3(3)),
+    the query read and the output written, and the table entries and lengths
+    that locate them:
 
         sum_s ctx_s * Hkv * d * 2 * e      K and V of valid tokens
       + 2 * S * Hq * d * e                 q read, out written

@@ -247,6 +247,8 @@ FULL = {
     "gqa": lambda: W.gqa(device="cuda"),
     "shared_prefix_p512": lambda: W.shared_prefix(prompt_len=512, suffix_max=512, device="cuda"),
     "shared_prefix_p520_cow": lambda: W.shared_prefix(prompt_len=520, suffix_max=0, device="cuda"),
+    "shared_prefix_p512_part256": lambda: W.shared_prefix(prompt_len=512, suffix_max=512, device="cuda",
+                                                          partition_size=256),
     "long_context_b8": lambda: W.long_context(block_size=8, device="cuda"),
     "long_context_b16": lambda: W.long_context(block_size=16, device="cuda"),
     "long_context_b32": lambda: W.long_context(block_size=32, device="cuda"),
@@ -302,11 +304,10 @@ def test_full_size(pa, name, call):
     untouched = torch.ones(step.num_blocks, dtype=torch.bool, device="cuda")
     untouched[idx] = False
     assert torch.equal(kc[untouched], pre_k[untouched]) and torch.equal(vc[untouched], pre_v[untouched])
-    # decode: sampled sequences (shortest, longest and random ones), every head
-    rng = np.random.default_rng(0)
+    # decode: every sequence, every head, against the oracle run one sequence at
+    # a time on the blocks it reads (the oracle redoes the step's copies and write)
     ctx = step.context_lens
-    seqs = sorted({int(np.argmin(ctx)), int(np.argmax(ctx))} |
-                  set(int(x) for x in rng.choice(step.num_seqs, size=min(4, step.num_seqs), replace=False)))
+    seqs = list(range(step.num_seqs))
     ref = oracle_outputs(step, seqs, pre_k, pre_v)
     got = f64(out)
     for s in seqs:
@@ -421,6 +422,67 @@ def test_packed_shared_prefix_units_are_bit_identical(pa, heads):
     out2, *_ = run_gpu(pa, plain)
     assert torch.equal(out, out2)
     assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, f"packed {heads}")
+
+
+SHARED_LAYOUTS = [
+    # (Hq, Hkv, samples): query columns per shared unit = samples x g, in column groups of 8
+    (32, 8, 8),    # g 4: 32 columns, 4 groups
+    (32, 8, 5),    # 20 columns, 3 groups
+    (32, 8, 3),    # 12 columns, 2 groups
+    (16, 8, 12),   # g 2: 24 columns
+    (8, 8, 32),    # g 1: 32 columns
+    (8, 8, 12),    # 12 columns
+    (64, 8, 4),    # g 8: 32 columns
+    (64, 8, 3),    # 24 columns
+    (24, 8, 7),    # g 3: 21 columns, sequences straddle column groups
+]
+
+
+@pytest.mark.parametrize("d,B,P", [(128, 16, 128), (64, 8, 64), (128, 32, 32)], ids=["d128_b16_p128", "d64_b8_p64",
+                                                                                    "d128_b32_p32"])
+@pytest.mark.parametrize("layout", SHARED_LAYOUTS, ids=lambda c: f"h{c[0]}x{c[1]}_s{c[2]}")
+def test_shared_units_of_every_width(pa, layout, d, B, P):
+    """Samples sharing whole partitions are served by units of up to 32 query
+    columns that read each shared tile once (one warp per column group, a ring
+    of tiles shared by the CTA).  The output equals, bit for bit, the same batch
+    with private copies of the blocks (units of one column group, each warp one
+    stream), and the oracle within tolerance."""
+    Hq, Hkv, samples = layout
+    step = W.shared_prefix(prompt_len=3 * P + 8, suffix_max=P + 5, prompts=2, samples=samples, device="cuda",
+                           partition_size=P, num_heads=Hq, num_kv_heads=Hkv, head_dim=d, block_size=B)
+    out, kc, vc, err, _ = run_gpu(pa, step)
+    assert err == 0
+    after = W.DecodeStep(**{**step.__dict__})
+    after.k_cache, after.v_cache = kc, vc
+    out2, *_ = run_gpu(pa, unshared_copy(after))
+    assert torch.equal(out, out2)
+    assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, f"shared {layout}")
+
+
+def test_bad_block_in_a_shared_partition(pa):
+    """A block id outside the pool inside a shared partition: flagged, its tokens
+    skipped by every sample (their value rows zeroed by the ring's issuer), and
+    the result equals, bit for bit, private copies with the same bad entry."""
+    step = W.shared_prefix(prompt_len=200, suffix_max=40, prompts=2, samples=8, device="cuda", partition_size=64,
+                           num_heads=32, num_kv_heads=8, head_dim=128, block_size=16)
+    out_ok, kc, vc, err, _ = run_gpu(pa, step)
+    assert err == 0
+    after = W.DecodeStep(**{**step.__dict__})
+    after.k_cache, after.v_cache = kc, vc
+    after.slot_mapping = np.full_like(step.slot_mapping, -1)
+    after.copy_pairs = np.zeros((0, 2), dtype=np.int64)
+    plain = unshared_copy(after)
+    bad = after.num_blocks + 3
+    shared_tables = after.block_tables.copy()
+    shared_tables[:, 5] = bad                  # logical block 5: inside the shared second partition
+    plain_tables = plain.block_tables.copy()
+    plain_tables[:, 5] = bad + plain.num_blocks
+    a, _, _, ea, _ = run_gpu(pa, after, tables=shared_tables)
+    b, _, _, eb, _ = run_gpu(pa, plain, tables=plain_tables)
+    assert ea & pa.DEVERR_BLOCK_ID and eb & pa.DEVERR_BLOCK_ID
+    assert torch.isfinite(a).all()
+    assert torch.equal(a, b)
+    assert not torch.equal(a, out_ok)
 
 
 def random_fork_step(seed, Hq, Hkv, d, B, P, adjacent=True):
@@ -702,6 +764,59 @@ def test_prefill_reservation_and_free_blocks_are_ignored(pa):
     assert ea == 0 and eb == 0
     assert torch.isfinite(b).all()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("where", ["value", "key"])
+def test_prefill_tensor_core_non_finite_visible_value(pa, where):
+    """The tensor-core prefill reads a tile's K/V once for all 128 query rows of a
+    unit (32 new tokens x 4 heads here), so a NaN value element at a visible
+    position t reaches that output column of every row of the unit holding t:
+    rows at positions >= t, as in plain attention, and also the unit's earlier
+    rows (the documented departure; their weight for t is 0, but 0 * NaN is
+    NaN).  A NaN key at t is masked per row before the softmax and reaches only
+    rows at positions >= t (all their columns).  Everything else matches the
+    oracle; other kv heads are untouched."""
+    cached, new, Hq, Hkv, d, B = 40, 100, 32, 8, 128, 16
+    case = ([cached + new], [new], Hq, Hkv, d, B, 64)
+    assert pa.prefill_uses_tensor_cores(torch.bfloat16, Hq, Hkv, d, B)
+    step, q, qs = prefill_inputs(case, torch.bfloat16)
+    ref_clean = oracle.prefill_attention(f64(q), f64(step.k_cache), f64(step.v_cache), step.block_tables,
+                                         step.context_lens, qs, step.scale)
+    t = 80                                     # a position inside the second unit (new tokens 32..63)
+    pool = step.v_cache if where == "value" else step.k_cache
+    pool[int(step.block_tables[0, t // B]), 0, t % B, 5] = float("nan")   # kv head 0 only
+    out, err = run_prefill(pa, step, q, qs)
+    assert err == 0
+    got = f64(out)
+    pos = cached + np.arange(new)
+    g = Hq // Hkv
+    tq = 128 // g                              # new tokens per unit
+    unit_last = np.minimum((np.arange(new) // tq + 1) * tq, new) - 1 + cached
+    for h in range(Hq):
+        if h >= g:                             # heads of the other kv heads: plain parity
+            assert_close(got[:, h], ref_clean[:, h], torch.bfloat16, torch.float32, f"head {h}")
+            continue
+        late = pos >= t
+        if where == "key":
+            # a NaN score: the whole row is NaN for every row that sees t, nothing else changes
+            assert not np.isfinite(got[late, h]).any(), "rows at or after the NaN key must be NaN"
+            clean = ~late
+            assert_close(got[clean, h], ref_clean[clean, h], torch.bfloat16, torch.float32, f"head {h}")
+            continue
+        # a NaN in value column e: column e is NaN for the rows at or after t and for
+        # the earlier rows of the unit holding t (0 * NaN inside the tile's P.V);
+        # every other element equals plain attention
+        e = 5
+        reached = (~late) & (unit_last >= t)
+        assert reached.sum() > 0
+        assert not np.isfinite(got[late, h, e]).any(), "column e of rows at or after t"
+        assert not np.isfinite(got[reached, h, e]).any(), "column e of the earlier rows of t's unit"
+        rest = ~(late | reached)
+        assert rest.sum() > 0
+        assert_close(got[rest, h], ref_clean[rest, h], torch.bfloat16, torch.float32, f"head {h} other rows")
+        cols = np.arange(d) != e
+        assert_close(got[~rest, h][:, cols], ref_clean[~rest, h][:, cols], torch.bfloat16, torch.float32,
+                     f"head {h} other columns")
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])

@@ -49,6 +49,26 @@ def test_library_exports_only_the_c_abi(pa):
     assert exported == set(declared_functions()), sorted(exported ^ set(declared_functions()))
 
 
+def test_noalloc_limit_matches_the_header(pa):
+    """The binding's copy of PA_NOALLOC_SCRATCH_BYTES is the header's value."""
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+PA_NOALLOC_SCRATCH_BYTES\s+\(([^)]*)\)", text)
+    assert m, "PA_NOALLOC_SCRATCH_BYTES not found in include/pa.h"
+    expr = re.sub(r"(\d+)[uUlL]+", r"\1", m.group(1))
+    assert re.fullmatch(r"[\d\s\*\+]+", expr), expr
+    assert eval(expr) == pa.NOALLOC_SCRATCH_BYTES
+
+
+def test_status_codes_match_the_header(pa):
+    text = open(HEADER).read()
+    for name in ["PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE", "PA_ERR_CUDA",
+                 "PA_ERR_DEVICE_INDEX"]:
+        m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
+        assert m, name
+        assert int(m.group(1)) == getattr(pa, name), name
+        assert name.encode() in pa.lib.pa_status_string(int(m.group(1)))
+
+
 def test_status_strings_and_version(pa):
     assert pa.lib.pa_status_string(0).decode() == "PA_OK"
     assert b"workspace" in pa.lib.pa_status_string(3)
