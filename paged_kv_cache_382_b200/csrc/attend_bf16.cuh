@@ -1,5 +1,6 @@
-// attend_bf16.cuh -- the bf16 decode-attention kernel: one unit is one
-// partition of one kv head, for up to 32 query columns that read it.
+// attend_bf16.cuh -- the bf16 decode-attention kernel's building blocks: one
+// unit is one partition of one kv head, for up to 8 query columns per warp of
+// the CTA that read it.
 //
 // What a unit computes ("PagedAttention blog" section 3(3) decode step;
 // "Month 2 · PagedAttention" section 06): for each of its query columns
@@ -11,8 +12,9 @@
 // consecutive sequences name the same physical blocks for the whole partition
 // (parallel samples sharing a prompt's blocks, "PagedAttention blog" section 4;
 // "Month 2 · PagedAttention" sections 02 and 04), the g heads of each of up to
-// 32 / g such sequences: one read of the shared blocks serves them all.  The
-// columns are split into column groups (cg) of 8, the N of one m16n8k16 MMA.
+// 8 W / g such sequences (W warps): one read of the shared blocks serves them
+// all.  The columns are split into column groups (cg) of 8, the N of one
+// m16n8k16 MMA.
 //
 // Streams.  Every column's softmax runs as W streams (stream s takes the
 // partition's 16-token tiles s, s + W, s + 2W, ...), merged in stream order at

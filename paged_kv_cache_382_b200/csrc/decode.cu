@@ -58,7 +58,7 @@ struct DecodeArgs {
     int* ws_count;       // [1]   number of work items
     unsigned long long* ws_ticket;   // [1] bf16 attend: units taken past the first grid-wide wave (0 after
                                      //     the plan; the last fetch of a launch sets it back to 0)
-    int* ws_items;       // [num_seqs * max_parts]  see make_item
+    int2* ws_items;      // [num_seqs * max_parts]  (make_item code, clamped context of its sequence)
     float2* ws_ml;       // [num_seqs][num_heads][max_parts]  (log2-domain max, sum)
     float* ws_acc;       // [num_seqs][num_heads][max_parts][head_dim]
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks;
@@ -143,25 +143,35 @@ __device__ int shared_lead(const DecodeArgs& a, int s, int c, int c_next, int fi
 // partition (consecutive links); a sequence not covered that way emits its
 // own item.  `lead` holds shared_lead of the sequences from lead_base on.
 template <bool WRITE>
-__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int c0, int* out) {
+__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int c0, int2* out) {
     const int nfull = c / a.partition_size, m = a.pack;
     if (m <= 1) {
         if (WRITE)
-            for (int k = 0; k < nfull; ++k) out[k] = make_item(s, k, 1, a.max_parts);
+            for (int k = 0; k < nfull; ++k) out[k] = make_int2(make_item(s, k, 1, a.max_parts), c);
         return nfull;
     }
-    const int j = s - c0;
-    const int end = min(c0 + m, min(a.num_seqs, lead_base + PLAN_THREADS));
-    int n = 0;
-    for (int k = 0; k < nfull; ++k) {
-        int cnt = 1;
-        while (c0 + cnt < end && lead[c0 + cnt - 1 - lead_base] > k) ++cnt;
-        if (j == 0 || j >= cnt) {
-            if (WRITE) out[n] = make_item(s, k, j == 0 ? cnt : 1, a.max_parts);
-            ++n;
+    const int end = min(c0 + m, min(a.num_seqs, lead_base + static_cast<int>(blockDim.x)));   // the run: [c0, end)
+    if (s == c0) {
+        // partitions shared with the next sequence of the run get one item for
+        // the run-mates linked through them; the rest are the run start's own
+        const int kshared = s + 1 < end ? min(nfull, lead[s - lead_base]) : 0;
+        if (WRITE) {
+            for (int k = 0; k < kshared; ++k) {
+                int cnt = 2;
+                while (c0 + cnt < end && lead[c0 + cnt - 1 - lead_base] > k) ++cnt;
+                out[k] = make_int2(make_item(s, k, cnt, a.max_parts), c);
+            }
+            for (int k = kshared; k < nfull; ++k) out[k] = make_int2(make_item(s, k, 1, a.max_parts), c);
         }
+        return nfull;
     }
-    return n;
+    // a later member is served by the run start's items for the partitions that
+    // every link from c0 to it shares; it emits its own items for the rest
+    int covered = nfull;
+    for (int t = c0; t < s && covered > 0; ++t) covered = min(covered, lead[t - lead_base]);
+    if (WRITE)
+        for (int k = covered; k < nfull; ++k) out[k - covered] = make_int2(make_item(s, k, 1, a.max_parts), c);
+    return nfull - covered;
 }
 
 // Start of s's packing run: runs of a.pack sequences counted from the start of
@@ -176,22 +186,34 @@ __device__ __forceinline__ int run_start(const DecodeArgs& a, int start, const i
     return start + chain + ((t - chain) / a.pack) * a.pack;
 }
 
-// The plan itself, run by one CTA of PLAN_THREADS threads.
+// The plan itself, run by one CTA; its threads take one sequence each, a chunk
+// of blockDim.x sequences at a time.
+// Ragged tails are emitted longest first, in TAIL_BUCKETS classes of length,
+// so that the units handed out last are the short ones.
+constexpr int TAIL_BUCKETS = 4;
+
+__device__ __forceinline__ int tail_bucket(int c, int P) {
+    const int len = c - (c / P) * P;   // 1..P-1 tokens; 0 for an empty context
+    return (len * TAIL_BUCKETS) / P;   // TAIL_BUCKETS - 1 = the longest
+}
+
 __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
     __shared__ int scratch[33];
     __shared__ int lead[PLAN_THREADS];
     if (threadIdx.x == 0) *a.ws_ticket = 0;
     const int P = a.partition_size;
-    // Sequences are taken PLAN_THREADS at a time (a multiple of every packing
-    // run length).  Items: whole partitions first, then one per ragged tail,
-    // then one per empty context (it writes zeros).  One pass when the batch
-    // fits one chunk; otherwise a counting pass, then a writing pass.
-    const bool one_chunk = a.num_seqs <= PLAN_THREADS;
-    int full_total = 0, tail_total = 0;
-    int c = 0, f = 0, t = 0, ef = 0, et = 0;
-    for (int start = 0; start < a.num_seqs; start += PLAN_THREADS) {
+    // Items: whole partitions first, then one per ragged tail (longest class
+    // first), then nothing else: an empty context is a tail of the shortest
+    // class (its unit writes zeros).  One pass when the batch fits one chunk;
+    // otherwise a counting pass, then a writing pass.
+    const int CH = blockDim.x;
+    const bool one_chunk = a.num_seqs <= CH;
+    int full_total = 0, tail_total[TAIL_BUCKETS] = {0, 0, 0, 0};
+    int c = 0, f = 0, tb = -1, ef = 0, et = 0;
+    for (int start = 0; start < a.num_seqs; start += CH) {
         const int s = start + threadIdx.x;
-        f = t = 0;
+        f = 0;
+        tb = -1;
         __syncthreads();
         if (s < a.num_seqs) {
             const bool has_next = s + 1 < a.num_seqs;
@@ -202,31 +224,47 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
             c = clamp_context(raw, a.cap);
             if (c != raw) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
             lead[threadIdx.x] = shared_lead(a, s, c, clamp_context(raw_next, a.cap), first, first_next);
-            t = (c % P) != 0 || c == 0;
+            if ((c % P) != 0 || c == 0) tb = tail_bucket(c, P);
         }
         __syncthreads();
         const int c0 = run_start(a, start, lead, scratch);
         if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, nullptr);
-        int cf = 0, ct = 0;
+        int cf = 0;
         ef = cta_exclusive_scan(f, &cf, scratch);
-        et = cta_exclusive_scan(t, &ct, scratch);
         full_total += cf;
-        tail_total += ct;
+#pragma unroll
+        for (int b = 0; b < TAIL_BUCKETS; ++b) {
+            int cb = 0;
+            const int eb = cta_exclusive_scan(tb == b, &cb, scratch);
+            if (tb == b) et = eb;
+            tail_total[b] += cb;
+        }
+    }
+    // first slot of each tail class, longest class first
+    int tail_base[TAIL_BUCKETS];
+    {
+        int acc = full_total;
+#pragma unroll
+        for (int b = TAIL_BUCKETS - 1; b >= 0; --b) {
+            tail_base[b] = acc;
+            acc += tail_total[b];
+        }
+        if (threadIdx.x == 0) *a.ws_count = acc;
     }
     if (one_chunk) {
         const int s = threadIdx.x;
         const int c0 = run_start(a, 0, lead, scratch);
         if (s < a.num_seqs) {
             full_items<true>(a, s, c, lead, 0, c0, a.ws_items + ef);
-            if (t) a.ws_items[full_total + et] = make_item(s, c / P, 1, a.max_parts);
+            if (tb >= 0) a.ws_items[tail_base[tb] + et] = make_int2(make_item(s, c / P, 1, a.max_parts), c);
         }
-        if (threadIdx.x == 0) *a.ws_count = full_total + tail_total;
         return;
     }
-    int base_full = 0, base_tail = full_total;
-    for (int start = 0; start < a.num_seqs; start += PLAN_THREADS) {
+    int base_full = 0;
+    for (int start = 0; start < a.num_seqs; start += CH) {
         const int s = start + threadIdx.x;
-        f = t = 0;
+        f = 0;
+        tb = -1;
         __syncthreads();
         if (s < a.num_seqs) {
             const bool has_next = s + 1 < a.num_seqs;
@@ -235,22 +273,23 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
             const int first = a.pack > 1 ? table_row(a, s)[0] : 0;
             const int first_next = (a.pack > 1 && has_next) ? table_row(a, s + 1)[0] : 1;
             lead[threadIdx.x] = shared_lead(a, s, c, c_next, first, first_next);
-            t = (c % P) != 0 || c == 0;
+            if ((c % P) != 0 || c == 0) tb = tail_bucket(c, P);
         }
         __syncthreads();
         const int c0 = run_start(a, start, lead, scratch);
         if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, nullptr);
-        int chunk_f = 0, chunk_t = 0;
+        int chunk_f = 0;
         ef = cta_exclusive_scan(f, &chunk_f, scratch);
-        et = cta_exclusive_scan(t, &chunk_t, scratch);
-        if (s < a.num_seqs) {
-            full_items<true>(a, s, c, lead, start, c0, a.ws_items + base_full + ef);
-            if (t) a.ws_items[base_tail + et] = make_item(s, c / P, 1, a.max_parts);
+        if (s < a.num_seqs) full_items<true>(a, s, c, lead, start, c0, a.ws_items + base_full + ef);
+#pragma unroll
+        for (int b = 0; b < TAIL_BUCKETS; ++b) {
+            int cb = 0;
+            const int eb = cta_exclusive_scan(tb == b, &cb, scratch);
+            if (tb == b) a.ws_items[tail_base[b] + eb] = make_int2(make_item(s, c / P, 1, a.max_parts), c);
+            tail_base[b] += cb;
         }
         base_full += chunk_f;
-        base_tail += chunk_t;
     }
-    if (threadIdx.x == 0) *a.ws_count = full_total + tail_total;
 }
 
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
@@ -337,9 +376,9 @@ __device__ __forceinline__ void combine_store(const DecodeArgs& a, const float* 
 // ---------------------------------------------------------------------------
 
 // Resident CTAs per SM the bf16 attend kernel is register-budgeted for (shared
-// memory allows 3 at 4 warps x 2 stages of 8 KB).
+// memory allows 4 at 3 warps x 2 stages of 8 KB).
 #ifndef PA_ATTEND_MIN_CTAS
-#define PA_ATTEND_MIN_CTAS 3
+#define PA_ATTEND_MIN_CTAS 4
 #endif
 
 // Stores a warp's final state of column group cg (columns 8cg .. 8cg+7) into
@@ -391,6 +430,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     __shared__ int s_abort;
     __shared__ int3 s_rows[32];
     __shared__ unsigned long long s_next;   // the next unit this CTA works on
+    __shared__ int2 s_next_item;            // and its work item
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -431,17 +471,20 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     // (whole partitions first), so a CTA that drew short units takes more.
     // Each fetch is made one unit ahead, its latency hidden behind the
     // current unit.
-    if (tid == 0) s_next = blockIdx.x;
+    if (tid == 0) {
+        s_next = blockIdx.x;
+        if (blockIdx.x < units) s_next_item = a.ws_items[blockIdx.x / per_item];
+    }
     __syncthreads();
     for (;;) {
         const long long u = static_cast<long long>(s_next);
         if (u >= units) break;
-        const int item = a.ws_items[u / per_item];
+        const int2 item = s_next_item;
         const int r = static_cast<int>(u % per_item);
         const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
         int s, p, count;
-        split_item(item, a.max_parts, s, p, count);
-        const int ctx = clamp_context(a.context_lens[s], a.cap);   // packed items: whole partitions
+        split_item(item.x, a.max_parts, s, p, count);
+        const int ctx = item.y;   // clamped by the plan; packed items: whole partitions
         const int t0 = p * P;
         const int t1 = min(t0 + P, ctx);
         const int ntok = t1 - t0;
@@ -451,19 +494,26 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
         __syncthreads();   // the previous unit's epilogue is done with shared memory; s_next read
         if (s_abort) break;
-        if (tid == 0) {   // the CTA's next unit
-            // One fetch per unit run, so fetch number units - 1 is the launch's
-            // last: it puts the ticket back for another launch over this plan.
+        // The CTA's next unit: one ticket fetch per unit run, so fetch number
+        // units - 1 is the launch's last and puts the ticket back for another
+        // launch over this plan.  Its result, the next item, and this unit's
+        // column rows reach shared memory only at the end of the unit, so no
+        // warp waits for them here.
+        unsigned long long next_u = 0;
+        int2 next_item = make_int2(0, 0);
+        if (tid == 0) {
             const unsigned long long v = atomicAdd(a.ws_ticket, 1ull);
             if (v + 1 == static_cast<unsigned long long>(units)) *a.ws_ticket = 0ull;
-            s_next = gridDim.x + v;
+            next_u = gridDim.x + v;
         }
+        int3 my_row = make_int3(0, 0, 0);
+        int my_ctx = 0;
         if (tid < 32) {
             int member, head;
             bool valid;
             unit_row(a, kvh, hg, count, tid, member, head, valid);
-            const int cm = valid ? clamp_context(a.context_lens[s + member], a.cap) : 0;
-            s_rows[tid] = make_int3(s + member, head, (cm + P - 1) / P);
+            my_ctx = valid ? (member == 0 ? ctx : a.context_lens[s + member]) : 0;
+            my_row = make_int3(s + member, head, 0);
         }
 
         // block-table slice of this partition, validated once and turned into
@@ -555,6 +605,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             };
             const int npro = my_tiles < NS ? my_tiles : NS;
             for (int j = 0; j < npro; ++j) issue(j);
+            // the next unit's item, loaded behind this unit's first copies
+            if (tid == 0 && next_u < static_cast<unsigned long long>(units)) next_item = a.ws_items[next_u / per_item];
             for (int j = 0; j < my_tiles; ++j) {
                 const int stage = static_cast<int>(n_used % NS);
                 const uint32_t parity = (n_used / NS) & 1u;
@@ -645,6 +697,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             if (tid == 0) {
                 const int npro = ntiles < CS ? ntiles : CS;
                 for (int k = 0; k < npro; ++k) issue_cta(k);
+                // the next unit's item, loaded behind this unit's first copies
+                if (next_u < static_cast<unsigned long long>(units)) next_item = a.ws_items[next_u / per_item];
             }
             if (warp < ncg) {
                 float* aslot = reinterpret_cast<float*>(stages + CS * STAGE + warp * SLOT_BYTES);
@@ -690,6 +744,15 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             ring_base += static_cast<uint32_t>(ntiles);
         }
 
+        if (tid == 0) {
+            s_next = next_u;
+            s_next_item = next_item;
+        }
+        if (tid < 32) {
+            const int cm = clamp_context(my_ctx, a.cap);
+            my_row.z = (cm + P - 1) / P;
+            s_rows[tid] = my_row;
+        }
         if (__syncthreads_or(failed)) {   // every warp is done with the stages either way
             if (tid == 0) {
                 flag_error(a.dev_err, PA_DEVERR_TIMEOUT);
@@ -712,43 +775,54 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             store_final<D>(S, fin_o, fin_ml, warp, g, c);
         }
         __syncthreads();
-        for (int idx = tid; idx < nrows * D; idx += W * 32) {
-            const int n = idx / D, d = idx - (idx / D) * D;
+        // four consecutive elements of one column per thread and step
+        for (int idx = tid; idx < nrows * (D / 4); idx += W * 32) {
+            const int n = idx / (D / 4), d0 = 4 * (idx - n * (D / 4));
             const int3 ri = s_rows[n];
-            float O;
+            float O[4];
             float2 ml;
             if (ncg == 1) {
-                // lane (g, c) holds columns 2c, 2c+1 and elements 16i + g (+8)
-                const int e = (n & 1) + 2 * ((d >> 3) & 1), i16 = d >> 4;
-                const int ol = 4 * (d & 7) + (n >> 1), sl = n >> 1;    // lane holding (n, d); a lane of column n
-                const int km = n & 1, ko = 4 + 4 * i16 + e;
+                // lane (g, c) holds columns 2c, 2c+1 and elements 16i + g (+8); the
+                // four elements sit in lanes 4g + c of one slot element each
+                const int e = (n & 1) + 2 * ((d0 >> 3) & 1), i16 = d0 >> 4;
+                const int sl = n >> 1, km = n & 1, ko = (4 + 4 * i16 + e) * 32 + sl;
                 float M = slots[km * 32 + sl], L = slots[(2 + km) * 32 + sl];
-                O = slots[ko * 32 + ol];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) O[k] = slots[ko + 4 * ((d0 + k) & 7)];
 #pragma unroll
                 for (int w = 1; w < W; ++w) {
                     const float* sw = slots + w * (SLOT_BYTES / 4);
                     float Mn, ca, cb;
                     merge_coef(M, sw[km * 32 + sl], Mn, ca, cb);
                     L = merge_val(ca, L, cb, sw[(2 + km) * 32 + sl]);
-                    O = merge_val(ca, O, cb, sw[ko * 32 + ol]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) O[k] = merge_val(ca, O[k], cb, sw[ko + 4 * ((d0 + k) & 7)]);
                     M = Mn;
                 }
                 ml = make_float2(M, L);
             } else {
-                O = fin_o[idx];
+                const float4 f = *reinterpret_cast<const float4*>(fin_o + n * D + d0);
+                O[0] = f.x;
+                O[1] = f.y;
+                O[2] = f.z;
+                O[3] = f.w;
                 ml = fin_ml[n];
             }
             const size_t row = static_cast<size_t>(ri.x) * a.num_heads + ri.y;
             if (ri.z <= 1) {
-                const float v = ml.y > 0.f ? O / ml.y : 0.f;
+                float v[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[k] = ml.y > 0.f ? O[k] / ml.y : 0.f;
                 if (a.out_f32)
-                    static_cast<float*>(a.out)[row * D + d] = v;
+                    *reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * D + d0) =
+                        make_float4(v[0], v[1], v[2], v[3]);
                 else
-                    static_cast<__nv_bfloat16*>(a.out)[row * D + d] = __float2bfloat16_rn(v);
+                    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + row * D + d0) =
+                        make_uint2(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]));
             } else {
                 const size_t slot = row * a.max_parts + p;
-                a.ws_acc[slot * D + d] = O;
-                if (d == 0) a.ws_ml[slot] = ml;
+                *reinterpret_cast<float4*>(a.ws_acc + slot * D + d0) = make_float4(O[0], O[1], O[2], O[3]);
+                if (d0 == 0) a.ws_ml[slot] = ml;
             }
         }
         fence_proxy_async_smem();   // these generic accesses precede the next unit's bulk copies
@@ -776,12 +850,12 @@ __global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) 
     const float* qp = static_cast<const float*>(a.q);
 
     for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-        const int item = a.ws_items[u / per_item];
+        const int2 item = a.ws_items[u / per_item];
         const int r = static_cast<int>(u % per_item);
         const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
         int s, p, count;
-        split_item(item, a.max_parts, s, p, count);   // this path is planned unpacked: count == 1
-        const int ctx = clamp_context(a.context_lens[s], a.cap);
+        split_item(item.x, a.max_parts, s, p, count);   // this path is planned unpacked: count == 1
+        const int ctx = item.y;
         const int t0 = p * P, t1 = min(t0 + P, ctx);
         const int nparts = (ctx + P - 1) / P;
         const int gsub = min(8, a.group - hg * 8);
@@ -870,7 +944,16 @@ __global__ void __launch_bounds__(128) reduce_heads_kernel(const DecodeArgs a) {
     const int nparts = (ctx + a.partition_size - 1) / a.partition_size;
     if (nparts <= 1 || head >= a.num_heads) return;   // single partitions are written by attend
     const size_t row = static_cast<size_t>(s) * a.num_heads + head;
+    const int c4 = lane % C4, sub = lane / C4;
+    const float4* accp = reinterpret_cast<const float4*>(a.ws_acc + row * a.max_parts * D) + c4;
+    // the (max, sum) pairs and the first batch of partials are loaded together
     const float2 ml = lane < nparts ? a.ws_ml[row * a.max_parts + lane] : make_float2(NEG_INF, 0.f);
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int p = u * SUB + sub;
+        if (p < nparts) v[u] = accp[static_cast<size_t>(p) * C4];
+    }
     float M = ml.x;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
@@ -878,15 +961,14 @@ __global__ void __launch_bounds__(128) reduce_heads_kernel(const DecodeArgs a) {
     float L = e * ml.y;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(FULL_MASK, L, off);
-    const int c4 = lane % C4, sub = lane / C4;
-    const float4* accp = reinterpret_cast<const float4*>(a.ws_acc + row * a.max_parts * D) + c4;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int p0 = 0; p0 < nparts; p0 += SUB * U) {
-        float4 v[U];
+        if (p0 > 0) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int p = p0 + u * SUB + sub;
-            if (p < nparts) v[u] = accp[static_cast<size_t>(p) * C4];
+            for (int u = 0; u < U; ++u) {
+                const int p = p0 + u * SUB + sub;
+                if (p < nparts) v[u] = accp[static_cast<size_t>(p) * C4];
+            }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -1026,7 +1108,7 @@ prefill_rows_kernel(const int32_t* __restrict__ context_lens, const int32_t* __r
 // ---------------------------------------------------------------------------
 
 #ifndef PA_ATTEND_WARPS
-#define PA_ATTEND_WARPS 4
+#define PA_ATTEND_WARPS 3
 #endif
 #ifndef PA_ATTEND_STAGES
 #define PA_ATTEND_STAGES 2
@@ -1044,7 +1126,7 @@ inline WsLayout ws_layout(int S, int Hq, int D, int max_parts) {
     WsLayout L;
     size_t off = 256;   // header: the work-item count (0) and the attend kernel's unit ticket (8)
     L.items = off;
-    off += round_up(static_cast<size_t>(S) * max_parts * sizeof(int), 256);
+    off += round_up(static_cast<size_t>(S) * max_parts * sizeof(int2), 256);
     if (max_parts > 1) {
         L.ml = off;
         off += round_up(static_cast<size_t>(S) * Hq * max_parts * sizeof(float2), 256);
@@ -1188,7 +1270,7 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     a.ws_count = reinterpret_cast<int*>(ws);
     a.ws_ticket = reinterpret_cast<unsigned long long*>(ws + 8);
-    a.ws_items = reinterpret_cast<int*>(ws + L.items);
+    a.ws_items = reinterpret_cast<int2*>(ws + L.items);
     a.ws_ml = max_parts > 1 ? reinterpret_cast<float2*>(ws + L.ml) : nullptr;
     a.ws_acc = max_parts > 1 ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
     a.num_seqs = num_seqs;
@@ -1216,10 +1298,13 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
 
     if (prep(st, a.cap) != PA_OK) return PA_ERR_CUDA;
     if (phases & PA_PHASE_PLAN) {
+        // one thread per sequence, in chunks of up to PLAN_THREADS; small batches
+        // take a small CTA (cheaper barriers in the plan's scans)
+        const int plan_threads = num_seqs >= PLAN_THREADS ? PLAN_THREADS : (num_seqs <= 128 ? 128 : (num_seqs + 31) / 32 * 32);
         const cudaError_t e =
             (scatter != nullptr && num_new_tokens > 0)
-                ? launch_pdl(step_prologue_kernel, dim3(1 + num_new_tokens), dim3(PLAN_THREADS), 0, st, a, *scatter)
-                : launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, st, a);
+                ? launch_pdl(step_prologue_kernel, dim3(1 + num_new_tokens), dim3(plan_threads), 0, st, a, *scatter)
+                : launch_pdl(plan_kernel, dim3(1), dim3(plan_threads), 0, st, a);
         if (launch_status(e) != PA_OK) return PA_ERR_CUDA;
     }
     if (phases & PA_PHASE_ATTEND) {

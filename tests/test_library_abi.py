@@ -108,14 +108,14 @@ def test_selftest_host_validation(pa):
 
 def test_workspace_bytes(pa):
     ws = pa.lib.pa_decode_workspace_bytes
-    # one partition: header + work list only
-    assert ws(64, 32, 128, 512, 512) == 256 + 256
+    # one partition: header + work list only (an item is two int32: code and context)
+    assert ws(64, 32, 128, 512, 512) == 256 + 512
     # several partitions: + (max, sum) and the fp32 partial outputs
     S, H, D, cap, P = 8, 64, 128, 131072, 512
     parts = cap // P
     r = lambda n: (n + 255) // 256 * 256  # noqa: E731
     # header, work list, (max, sum), partial outputs
-    expect = 256 + r(S * parts * 4) + r(S * H * parts * 8) + r(S * H * parts * D * 4)
+    expect = 256 + r(S * parts * 8) + r(S * H * parts * 8) + r(S * H * parts * D * 4)
     assert ws(S, H, D, cap, P) == expect
     assert ws(-1, 1, 64, 10, 512) == 0
     assert ws(1, 1, 64, 10, 0) == 0
