@@ -65,10 +65,8 @@ CONFIGS = {
                           desc="parallel sampling bf16: 16 prompts x 8 samples, 512-token prompt in "
                                "shared blocks, suffix uniform [0, 512], 32 q / 8 kv heads, head_dim 128"),
     "shared_prefix_cow": dict(max_len=521, builder="shared_prefix", kwargs=dict(prompt_len=520, suffix_max=0),
-                              partition_size=256,
                               desc="parallel sampling bf16, first decode step after a 520-token prompt: "
-                                   "112 copy-on-write block copies, 32 q / 8 kv heads, head_dim 128, "
-                                   "partitions of 256 tokens"),
+                                   "112 copy-on-write block copies, 32 q / 8 kv heads, head_dim 128"),
     "long_context_b8": dict(max_len=131072, builder="long_context", kwargs=dict(block_size=8),
                             desc="long-context decode bf16: 8 seqs, context lens uniform [32768, 131072], "
                                  "64 q / 8 kv heads, head_dim 128, block_size 8, partitions of 512"),

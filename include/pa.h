@@ -114,9 +114,12 @@ PA_API int pa_reshape_and_cache(const void* key, const void* value, void* k_cach
  * a batch of num_seqs sequences whose contexts do not exceed max_context_len,
  * split into partitions of partition_size tokens.  Returns 0 on bad arguments.
  * The workspace holds the per-call work list (num_seqs * ceil(max_context_len /
- * partition_size) entries) and, when a context can span several partitions,
- * one (max, sum, unnormalised output) partial per sequence, head and partition
- * in fp32.  Its contents need no initialisation.
+ * partition_size) entries of 16 bytes, plus room for the extra items of split
+ * shared partitions), when a context can span several partitions one (max,
+ * sum, unnormalised output) partial per sequence, head and partition in fp32,
+ * and the per-stream states of up to 256 shared units (one kv head of a
+ * partition that several sequences name) whose streams run on separate CTAs.
+ * Its contents need no initialisation.
  */
 PA_API size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                  int max_context_len, int partition_size);
@@ -146,6 +149,10 @@ PA_API size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_di
  * carried to about 16 significant bits into the value product; fp32 inputs: fp32
  * throughout.  The result depends only on the logical order of the tokens, so it is
  * bit-identical under any renumbering of physical blocks and run to run.
+ * Sequences whose block tables name the same physical blocks for a whole partition
+ * (parallel samples of one prompt, prefix-cached requests) are served together, the
+ * shared blocks read once for all of them (bf16, up to 24 / g sequences per read);
+ * their outputs are bit-identical to those of private copies of the blocks.
  * Launches three kernels (plan, attention, merge) on `stream`.
  */
 PA_API int pa_decode(void* out, pa_dtype out_dtype, const void* q, const void* k_cache,

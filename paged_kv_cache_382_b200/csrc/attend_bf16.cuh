@@ -140,6 +140,40 @@ __device__ __forceinline__ void merge_slot_first(StreamState<D>& R, const float*
     }
 }
 
+// R = R (A, earlier) merged with the state at g (B, later), a state another
+// CTA wrote to global memory (read from L2, past this SM's L1).
+template <int D>
+__device__ __forceinline__ void merge_global_second(StreamState<D>& R, const float* g, int lane) {
+    float M0, M1, a0, a1, b0, b1;
+    merge_coef(R.m0, __ldcg(g + 0 * 32 + lane), M0, a0, b0);
+    merge_coef(R.m1, __ldcg(g + 1 * 32 + lane), M1, a1, b1);
+    R.m0 = M0;
+    R.m1 = M1;
+    R.l0 = merge_val(a0, R.l0, b0, __ldcg(g + 2 * 32 + lane));
+    R.l1 = merge_val(a1, R.l1, b1, __ldcg(g + 3 * 32 + lane));
+#pragma unroll
+    for (int i = 0; i < StreamState<D>::KS; ++i) {
+        const float* go = g + (4 + 4 * i) * 32 + lane;
+        R.o[i][0] = merge_val(a0, R.o[i][0], b0, __ldcg(go + 0 * 32));
+        R.o[i][1] = merge_val(a1, R.o[i][1], b1, __ldcg(go + 1 * 32));
+        R.o[i][2] = merge_val(a0, R.o[i][2], b0, __ldcg(go + 2 * 32));
+        R.o[i][3] = merge_val(a1, R.o[i][3], b1, __ldcg(go + 3 * 32));
+    }
+}
+
+// R = the state at g (written by another CTA; read from L2).
+template <int D>
+__device__ __forceinline__ void load_global_state(StreamState<D>& R, const float* g, int lane) {
+    R.m0 = __ldcg(g + 0 * 32 + lane);
+    R.m1 = __ldcg(g + 1 * 32 + lane);
+    R.l0 = __ldcg(g + 2 * 32 + lane);
+    R.l1 = __ldcg(g + 3 * 32 + lane);
+#pragma unroll
+    for (int i = 0; i < StreamState<D>::KS; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) R.o[i][e] = __ldcg(g + (4 + 4 * i + e) * 32 + lane);
+}
+
 // slot (A, earlier) = slot merged with R (B, later).
 template <int D>
 __device__ __forceinline__ void merge_into_slot(float* slot, const StreamState<D>& R, int lane) {

@@ -46,6 +46,17 @@
 
 namespace pa {
 
+#ifndef PA_ATTEND_WARPS
+#define PA_ATTEND_WARPS 3
+#endif
+#ifndef PA_ATTEND_STAGES
+#define PA_ATTEND_STAGES 2
+#endif
+constexpr int ATTEND_WARPS = PA_ATTEND_WARPS;    // warps per CTA of the bf16 attend kernel
+constexpr int ATTEND_STAGES = PA_ATTEND_STAGES;  // ring stages per warp
+constexpr int ATTEND_STREAMS = ATTEND_WARPS;     // softmax streams per query column
+// split shared units (item x kv head) whose stream states the workspace holds
+constexpr int SPLIT_CAP_MAX = 256;
 
 struct DecodeArgs {
     void* out;
@@ -58,7 +69,12 @@ struct DecodeArgs {
     int* ws_count;       // [1]   number of work items
     unsigned long long* ws_ticket;   // [1] bf16 attend: units taken past the first grid-wide wave (0 after
                                      //     the plan; the last fetch of a launch sets it back to 0)
-    int2* ws_items;      // [num_seqs * max_parts]  (make_item code, clamped context of its sequence)
+    int4* ws_items;      // [item capacity]  (make_item code, clamped context of its sequence,
+                         //                   split slot of kv head 0 or -1, unused)
+    float* ws_split;     // [split_cap][W streams][W column groups][state]  stream states of split shared units
+    int* ws_split_cnt;   // [split_cap]  streams finished per split unit (0 between launches)
+    int split_cap;       // split units (item x kv head) the workspace holds
+    int split_items;     // shared items the plan may split: split_cap / num_kv_heads
     float2* ws_ml;       // [num_seqs][num_heads][max_parts]  (log2-domain max, sum)
     float* ws_acc;       // [num_seqs][num_heads][max_parts][head_dim]
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks;
@@ -80,16 +96,20 @@ __device__ __forceinline__ const int32_t* table_row(const DecodeArgs& a, int s) 
     return a.block_tables + static_cast<size_t>(a.row_seq != nullptr ? a.row_seq[s] : s) * a.max_blocks;
 }
 
-// A work item names a partition p of sequence s and how many consecutive
+// A work item names a partition p of sequence s, how many consecutive
 // sequences (s, s+1, ..., at most 32) share that partition's blocks and are
-// served by it.
+// served by it, and, for a shared partition whose streams are split over
+// several CTAs, which stream this item runs.
 constexpr int ITEM_COUNT_BITS = 5;
-__host__ __device__ __forceinline__ int make_item(int s, int p, int count, int max_parts) {
-    return ((s * max_parts + p) << ITEM_COUNT_BITS) | (count - 1);
+constexpr int ITEM_STREAM_BITS = 2;
+constexpr int ITEM_LOW_BITS = ITEM_COUNT_BITS + ITEM_STREAM_BITS;
+__host__ __device__ __forceinline__ int make_item(int s, int p, int count, int max_parts, int stream = 0) {
+    return ((s * max_parts + p) << ITEM_LOW_BITS) | (stream << ITEM_COUNT_BITS) | (count - 1);
 }
-__device__ __forceinline__ void split_item(int item, int max_parts, int& s, int& p, int& count) {
+__device__ __forceinline__ void split_item(int item, int max_parts, int& s, int& p, int& count, int& stream) {
     count = (item & ((1 << ITEM_COUNT_BITS) - 1)) + 1;
-    const int sp = item >> ITEM_COUNT_BITS;
+    stream = (item >> ITEM_COUNT_BITS) & ((1 << ITEM_STREAM_BITS) - 1);
+    const int sp = item >> ITEM_LOW_BITS;
     s = sp / max_parts;
     p = sp - s * max_parts;
 }
@@ -142,35 +162,79 @@ __device__ int shared_lead(const DecodeArgs& a, int s, int c, int c_next, int fi
 // first sequence emits one item for the run-mates linked to it through that
 // partition (consecutive links); a sequence not covered that way emits its
 // own item.  `lead` holds shared_lead of the sequences from lead_base on.
+// Query columns of a packed item of `count` sequences: it takes the CTA-wide
+// shared layout (several column groups) when they exceed one group of 8.
+__device__ __forceinline__ bool shared_layout(const DecodeArgs& a, int count) { return count * a.group > 8; }
+
+// Number of consecutive sequences from c0 (at most the run's end) linked to c0
+// through partition k.
+__device__ __forceinline__ int run_count(const int* lead, int lead_base, int c0, int end, int k) {
+    int cnt = 2;
+    while (c0 + cnt < end && lead[c0 + cnt - 1 - lead_base] > k) ++cnt;
+    return cnt;
+}
+
+// Shared items of the shared layout that sequence s starts (candidates for a
+// split over CTAs, numbered by the plan across the batch).
+__device__ int split_candidates(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int c0) {
+    if (a.pack <= 1 || s != c0 || a.split_items <= 0) return 0;
+    const int end = min(c0 + a.pack, min(a.num_seqs, lead_base + static_cast<int>(blockDim.x)));
+    const int kshared = s + 1 < end ? min(c / a.partition_size, lead[s - lead_base]) : 0;
+    int n = 0;
+    for (int k = 0; k < kshared; ++k) n += shared_layout(a, run_count(lead, lead_base, c0, end, k));
+    return n;
+}
+
+// Whole-partition items of sequence s (context c), counted or written to out[].
+// Sequences are packed in runs of up to a.pack, aligned at the start of each
+// chain of consecutive sequences that share their first partition (c0 is the
+// start of s's run) and cut at the chunk's end: for each partition, the run's
+// first sequence emits one item for the run-mates linked to it through that
+// partition (consecutive links); a sequence not covered that way emits its
+// own item.  A shared-layout item whose number (split_id, counted over the
+// batch) is below a.split_items is emitted as W items, one per stream, that
+// run on different CTAs.  `lead` holds shared_lead of the sequences from
+// lead_base on.
 template <bool WRITE>
-__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int c0, int2* out) {
+__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int c0, int split_id,
+                          int4* out) {
     const int nfull = c / a.partition_size, m = a.pack;
     if (m <= 1) {
         if (WRITE)
-            for (int k = 0; k < nfull; ++k) out[k] = make_int2(make_item(s, k, 1, a.max_parts), c);
+            for (int k = 0; k < nfull; ++k) out[k] = make_int4(make_item(s, k, 1, a.max_parts), c, -1, 0);
         return nfull;
     }
     const int end = min(c0 + m, min(a.num_seqs, lead_base + static_cast<int>(blockDim.x)));   // the run: [c0, end)
     if (s == c0) {
-        // partitions shared with the next sequence of the run get one item for
-        // the run-mates linked through them; the rest are the run start's own
+        // partitions shared with the next sequence of the run get one item (or
+        // one per stream) for the run-mates linked through them; the rest are
+        // the run start's own
         const int kshared = s + 1 < end ? min(nfull, lead[s - lead_base]) : 0;
-        if (WRITE) {
-            for (int k = 0; k < kshared; ++k) {
-                int cnt = 2;
-                while (c0 + cnt < end && lead[c0 + cnt - 1 - lead_base] > k) ++cnt;
-                out[k] = make_int2(make_item(s, k, cnt, a.max_parts), c);
+        int n = 0;
+        for (int k = 0; k < kshared; ++k) {
+            const int cnt = run_count(lead, lead_base, c0, end, k);
+            if (shared_layout(a, cnt) && split_id < a.split_items) {
+                if (WRITE)
+                    for (int st = 0; st < ATTEND_STREAMS; ++st)
+                        out[n + st] = make_int4(make_item(s, k, cnt, a.max_parts, st), c, split_id * a.num_kv_heads, 0);
+                n += ATTEND_STREAMS;
+                ++split_id;
+                continue;
             }
-            for (int k = kshared; k < nfull; ++k) out[k] = make_int2(make_item(s, k, 1, a.max_parts), c);
+            if (shared_layout(a, cnt)) ++split_id;
+            if (WRITE) out[n] = make_int4(make_item(s, k, cnt, a.max_parts), c, -1, 0);
+            ++n;
         }
-        return nfull;
+        if (WRITE)
+            for (int k = kshared; k < nfull; ++k) out[n + k - kshared] = make_int4(make_item(s, k, 1, a.max_parts), c, -1, 0);
+        return n + nfull - kshared;
     }
     // a later member is served by the run start's items for the partitions that
     // every link from c0 to it shares; it emits its own items for the rest
     int covered = nfull;
     for (int t = c0; t < s && covered > 0; ++t) covered = min(covered, lead[t - lead_base]);
     if (WRITE)
-        for (int k = covered; k < nfull; ++k) out[k - covered] = make_int2(make_item(s, k, 1, a.max_parts), c);
+        for (int k = covered; k < nfull; ++k) out[k - covered] = make_int4(make_item(s, k, 1, a.max_parts), c, -1, 0);
     return nfull - covered;
 }
 
@@ -209,7 +273,9 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
     const int CH = blockDim.x;
     const bool one_chunk = a.num_seqs <= CH;
     int full_total = 0, tail_total[TAIL_BUCKETS] = {0, 0, 0, 0};
-    int c = 0, f = 0, tb = -1, ef = 0, et = 0;
+    int c = 0, f = 0, tb = -1, ef = 0, et = 0, sid = 0, split_total = 0;
+    // split units' counters start at zero (the last stream of a unit also resets its own)
+    for (int i = threadIdx.x; i < a.split_cap; i += blockDim.x) a.ws_split_cnt[i] = 0;
     for (int start = 0; start < a.num_seqs; start += CH) {
         const int s = start + threadIdx.x;
         f = 0;
@@ -228,7 +294,11 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
         }
         __syncthreads();
         const int c0 = run_start(a, start, lead, scratch);
-        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, nullptr);
+        int nsplit = 0;
+        sid = split_total + cta_exclusive_scan(s < a.num_seqs ? split_candidates(a, s, c, lead, start, c0) : 0,
+                                               &nsplit, scratch);
+        split_total += nsplit;
+        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, sid, nullptr);
         int cf = 0;
         ef = cta_exclusive_scan(f, &cf, scratch);
         full_total += cf;
@@ -255,12 +325,13 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
         const int s = threadIdx.x;
         const int c0 = run_start(a, 0, lead, scratch);
         if (s < a.num_seqs) {
-            full_items<true>(a, s, c, lead, 0, c0, a.ws_items + ef);
-            if (tb >= 0) a.ws_items[tail_base[tb] + et] = make_int2(make_item(s, c / P, 1, a.max_parts), c);
+            full_items<true>(a, s, c, lead, 0, c0, sid, a.ws_items + ef);
+            if (tb >= 0) a.ws_items[tail_base[tb] + et] = make_int4(make_item(s, c / P, 1, a.max_parts), c, -1, 0);
         }
         return;
     }
     int base_full = 0;
+    split_total = 0;
     for (int start = 0; start < a.num_seqs; start += CH) {
         const int s = start + threadIdx.x;
         f = 0;
@@ -277,15 +348,19 @@ __device__ __forceinline__ void plan_body(const DecodeArgs& a) {
         }
         __syncthreads();
         const int c0 = run_start(a, start, lead, scratch);
-        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, nullptr);
+        int nsplit = 0;
+        sid = split_total + cta_exclusive_scan(s < a.num_seqs ? split_candidates(a, s, c, lead, start, c0) : 0,
+                                               &nsplit, scratch);
+        split_total += nsplit;
+        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, sid, nullptr);
         int chunk_f = 0;
         ef = cta_exclusive_scan(f, &chunk_f, scratch);
-        if (s < a.num_seqs) full_items<true>(a, s, c, lead, start, c0, a.ws_items + base_full + ef);
+        if (s < a.num_seqs) full_items<true>(a, s, c, lead, start, c0, sid, a.ws_items + base_full + ef);
 #pragma unroll
         for (int b = 0; b < TAIL_BUCKETS; ++b) {
             int cb = 0;
             const int eb = cta_exclusive_scan(tb == b, &cb, scratch);
-            if (tb == b) a.ws_items[tail_base[b] + eb] = make_int2(make_item(s, c / P, 1, a.max_parts), c);
+            if (tb == b) a.ws_items[tail_base[b] + eb] = make_int4(make_item(s, c / P, 1, a.max_parts), c, -1, 0);
             tail_base[b] += cb;
         }
         base_full += chunk_f;
@@ -430,7 +505,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     __shared__ int s_abort;
     __shared__ int3 s_rows[32];
     __shared__ unsigned long long s_next;   // the next unit this CTA works on
-    __shared__ int2 s_next_item;            // and its work item
+    __shared__ int4 s_next_item;            // and its work item
+    __shared__ int s_last;                  // split units: this CTA finished the unit's last stream
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -479,11 +555,12 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     for (;;) {
         const long long u = static_cast<long long>(s_next);
         if (u >= units) break;
-        const int2 item = s_next_item;
+        const int4 item = s_next_item;
         const int r = static_cast<int>(u % per_item);
         const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
-        int s, p, count;
-        split_item(item.x, a.max_parts, s, p, count);
+        int s, p, count, stream;
+        split_item(item.x, a.max_parts, s, p, count, stream);
+        const int split_slot = item.z >= 0 ? item.z + kvh : -1;   // a split shared unit: this CTA runs one stream
         const int ctx = item.y;   // clamped by the plan; packed items: whole partitions
         const int t0 = p * P;
         const int t1 = min(t0 + P, ctx);
@@ -500,7 +577,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         // column rows reach shared memory only at the end of the unit, so no
         // warp waits for them here.
         unsigned long long next_u = 0;
-        int2 next_item = make_int2(0, 0);
+        int4 next_item = make_int4(0, 0, -1, 0);
         if (tid == 0) {
             const unsigned long long v = atomicAdd(a.ws_ticket, 1ull);
             if (v + 1 == static_cast<unsigned long long>(units)) *a.ws_ticket = 0ull;
@@ -531,11 +608,17 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         const int ntiles = (ntok + 15) / 16;
         const int qn = ntiles / W, rem = ntiles - qn * W;   // streams 0..rem-1 hold qn + 1 tiles
+        // positions of the CTA ring: the tiles in stream order (stream 0's, then
+        // stream 1's, ...), or only this CTA's stream for a split unit
+        const int npos = split_slot >= 0 ? (stream < rem ? qn + 1 : qn) : ntiles;
         if (ncg > 1) {
-            // the CTA ring passes the tiles in stream order: stream 0's, then stream 1's, ...
-            for (int j = tid; j < ntiles; j += W * 32) {
-                const int sj = j % W, tj = j / W;
-                ring_tile[sj * qn + min(sj, rem) + tj] = static_cast<uint16_t>(j);
+            if (split_slot >= 0) {
+                for (int k = tid; k < npos; k += W * 32) ring_tile[k] = static_cast<uint16_t>(stream + W * k);
+            } else {
+                for (int j = tid; j < ntiles; j += W * 32) {
+                    const int sj = j % W, tj = j / W;
+                    ring_tile[sj * qn + min(sj, rem) + tj] = static_cast<uint16_t>(j);
+                }
             }
         }
         // q fragments (B operand of S^T = K Q^T) of the lane's column g of its
@@ -695,7 +778,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 }
             };
             if (tid == 0) {
-                const int npro = ntiles < CS ? ntiles : CS;
+                const int npro = npos < CS ? npos : CS;
                 for (int k = 0; k < npro; ++k) issue_cta(k);
                 // the next unit's item, loaded behind this unit's first copies
                 if (next_u < static_cast<unsigned long long>(units)) next_item = a.ws_items[next_u / per_item];
@@ -703,8 +786,9 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             if (warp < ncg) {
                 float* aslot = reinterpret_cast<float*>(stages + CS * STAGE + warp * SLOT_BYTES);
                 int k = 0;
-                for (int sidx = 0; sidx < W; ++sidx) {
-                    if (sidx > 0) S.reset();
+                const int s_first = split_slot >= 0 ? stream : 0, s_end = split_slot >= 0 ? stream + 1 : W;
+                for (int sidx = s_first; sidx < s_end; ++sidx) {
+                    if (sidx > s_first) S.reset();
                     const int cnt = sidx < rem ? qn + 1 : qn;
                     for (int t = 0; t < cnt; ++t, ++k) {
                         const uint32_t pos = ring_base + static_cast<uint32_t>(k);
@@ -726,11 +810,18 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         // count); the last of the ncg readers refills it
                         if (lane == 0 && atomic_add_acq_rel_cta(&ccnt[stage], 1) == ncg - 1) {
                             ccnt[stage] = 0;
-                            if (k + CS < ntiles) issue_cta(k + CS);
+                            if (k + CS < npos) issue_cta(k + CS);
                         }
                     }
                     if (failed) break;
                     S.reduce_sums();
+                    if (split_slot >= 0) {
+                        // this CTA's stream of a split unit: its state goes to the
+                        // workspace; the CTA that finishes the unit's last stream merges
+                        S.store(a.ws_split + ((static_cast<size_t>(split_slot) * W + stream) * W + warp) *
+                                                 (State::FLOATS * 32), lane);
+                        break;
+                    }
                     // streams merge in order: slot = s0, then slot (+) s1, (+) s2; the
                     // last stream's merge leaves the column group's final state in S
                     if (sidx == 0)
@@ -741,7 +832,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         merge_slot_first<D>(S, aslot, lane);
                 }
             }
-            ring_base += static_cast<uint32_t>(ntiles);
+            ring_base += static_cast<uint32_t>(npos);
         }
 
         if (tid == 0) {
@@ -766,6 +857,28 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             break;
         }
         const float* slots = reinterpret_cast<const float*>(stages);
+        if (split_slot >= 0) {
+            // every stream's state is in the workspace once all W CTAs have counted
+            // themselves; the last one merges them in stream order (the merge of
+            // merge_into_slot / merge_slot_first) and writes the unit's outputs
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) {
+                const int done = atomicAdd(a.ws_split_cnt + split_slot, 1);
+                s_last = done == W - 1;
+                if (s_last) a.ws_split_cnt[split_slot] = 0;   // ready for another launch over this plan
+            }
+            __syncthreads();
+            if (!s_last) continue;
+            __threadfence();
+            if (warp < ncg) {
+                const float* st0 = a.ws_split + (static_cast<size_t>(split_slot) * W * W + warp) * (State::FLOATS * 32);
+                load_global_state<D>(S, st0, lane);
+#pragma unroll
+                for (int sidx = 1; sidx < W; ++sidx)
+                    merge_global_second<D>(S, st0 + static_cast<size_t>(sidx) * W * (State::FLOATS * 32), lane);
+            }
+        }
         if (ncg == 1) {
             // the W stream states wait in slots; every thread merges some of the
             // unit's (column, element) pairs, streams in order (the arithmetic of
@@ -850,11 +963,11 @@ __global__ void __launch_bounds__(128, 2) attend_f32_kernel(const DecodeArgs a) 
     const float* qp = static_cast<const float*>(a.q);
 
     for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-        const int2 item = a.ws_items[u / per_item];
+        const int4 item = a.ws_items[u / per_item];
         const int r = static_cast<int>(u % per_item);
         const int kvh = r / a.head_groups, hg = r - (r / a.head_groups) * a.head_groups;
-        int s, p, count;
-        split_item(item.x, a.max_parts, s, p, count);   // this path is planned unpacked: count == 1
+        int s, p, count, stream;
+        split_item(item.x, a.max_parts, s, p, count, stream);   // this path is planned unpacked: count == 1
         const int ctx = item.y;
         const int t0 = p * P, t1 = min(t0 + P, ctx);
         const int nparts = (ctx + P - 1) / P;
@@ -1107,26 +1220,29 @@ prefill_rows_kernel(const int32_t* __restrict__ context_lens, const int32_t* __r
 // host side
 // ---------------------------------------------------------------------------
 
-#ifndef PA_ATTEND_WARPS
-#define PA_ATTEND_WARPS 3
-#endif
-#ifndef PA_ATTEND_STAGES
-#define PA_ATTEND_STAGES 2
-#endif
-constexpr int ATTEND_WARPS = PA_ATTEND_WARPS;    // warps per CTA of the bf16 attend kernel
-constexpr int ATTEND_STAGES = PA_ATTEND_STAGES;  // ring stages per warp
 
 inline size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
 struct WsLayout {
-    size_t items, ml, acc, total;
+    size_t items, ml, acc, split, split_cnt, total;
+    int split_cap;
 };
+
+// Stream states of split shared units: a bounded number of (item, kv head)
+// units, at most one per two sequences, partition and query head.
+inline int split_cap_for(int S, int Hq, int max_parts) {
+    const long long bound = static_cast<long long>(S / 2) * max_parts * Hq;
+    return static_cast<int>(bound < SPLIT_CAP_MAX ? bound : SPLIT_CAP_MAX);
+}
 
 inline WsLayout ws_layout(int S, int Hq, int D, int max_parts) {
     WsLayout L;
+    L.split_cap = split_cap_for(S, Hq, max_parts);
     size_t off = 256;   // header: the work-item count (0) and the attend kernel's unit ticket (8)
     L.items = off;
-    off += round_up(static_cast<size_t>(S) * max_parts * sizeof(int2), 256);
+    // every (sequence, partition) item, plus W - 1 more for each split one
+    off += round_up((static_cast<size_t>(S) * max_parts + static_cast<size_t>(ATTEND_STREAMS - 1) * L.split_cap) *
+                        sizeof(int4), 256);
     if (max_parts > 1) {
         L.ml = off;
         off += round_up(static_cast<size_t>(S) * Hq * max_parts * sizeof(float2), 256);
@@ -1135,6 +1251,11 @@ inline WsLayout ws_layout(int S, int Hq, int D, int max_parts) {
     } else {
         L.ml = L.acc = 0;
     }
+    L.split = off;
+    off += round_up(static_cast<size_t>(L.split_cap) * ATTEND_STREAMS * ATTEND_WARPS * (4 * (D / 16) + 4) * 32 *
+                        sizeof(float), 256);
+    L.split_cnt = off;
+    off += round_up(static_cast<size_t>(L.split_cap) * sizeof(int), 256);
     L.total = off;
     return L;
 }
@@ -1244,7 +1365,7 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
 
     const long long cap = context_cap(max_blocks_per_seq, block_size, max_context_len);
     const int max_parts = parts_for(static_cast<int>(cap), partition_size);
-    if (static_cast<long long>(num_seqs) * max_parts > (INT_MAX >> ITEM_COUNT_BITS)) return PA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(num_seqs) * max_parts > (INT_MAX >> ITEM_LOW_BITS)) return PA_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, max_parts);
     if (!workspace || !aligned_to(workspace, 256)) return PA_ERR_INVALID_ARG;
     if (workspace_bytes < L.total) return PA_ERR_WORKSPACE;
@@ -1270,7 +1391,10 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     a.ws_count = reinterpret_cast<int*>(ws);
     a.ws_ticket = reinterpret_cast<unsigned long long*>(ws + 8);
-    a.ws_items = reinterpret_cast<int2*>(ws + L.items);
+    a.ws_items = reinterpret_cast<int4*>(ws + L.items);
+    a.ws_split = reinterpret_cast<float*>(ws + L.split);
+    a.ws_split_cnt = reinterpret_cast<int*>(ws + L.split_cnt);
+    a.split_cap = L.split_cap;
     a.ws_ml = max_parts > 1 ? reinterpret_cast<float2*>(ws + L.ml) : nullptr;
     a.ws_acc = max_parts > 1 ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
     a.num_seqs = num_seqs;
@@ -1293,6 +1417,7 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
     // group sequences sharing a partition's blocks share one unit (fp32 units
     // are never packed)
     a.pack = (dtype == PA_BF16 && a.group <= 8) ? 8 * ATTEND_WARPS / a.group : 1;
+    a.split_items = a.pack > 1 ? L.split_cap / num_kv_heads : 0;
     const cudaStream_t st = as_stream(stream);
     if (const int rc = device_check((phases & PA_PHASE_ATTEND) ? k_cache : context_lens)) return rc;
 

@@ -459,6 +459,45 @@ def test_shared_units_of_every_width(pa, layout, d, B, P):
     assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, f"shared {layout}")
 
 
+def test_shared_units_beyond_the_split_capacity(pa):
+    """More shared partitions than the workspace holds split units for (256 units
+    of one kv head): the first ones run as W stream units on different CTAs,
+    merged by the last, the rest as one CTA; all bit-identical to private copies
+    and within tolerance of the oracle."""
+    step = W.shared_prefix(prompt_len=64 * 3, suffix_max=20, prompts=16, samples=6, device="cuda",
+                           partition_size=64, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16)
+    # 16 prompts x 3 shared partitions = 48 shared items x 8 kv heads = 384 units > 256
+    out, kc, vc, err, _ = run_gpu(pa, step)
+    assert err == 0
+    after = W.DecodeStep(**{**step.__dict__})
+    after.k_cache, after.v_cache = kc, vc
+    out2, *_ = run_gpu(pa, unshared_copy(after))
+    assert torch.equal(out, out2)
+    assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.float32, "beyond the split capacity")
+
+
+def test_split_units_repeat_over_one_plan(pa):
+    """Split shared units count their finished streams in the workspace; the last
+    one resets the count, so attend + reduce run twice over one plan give the
+    whole call's result bit for bit both times."""
+    step = W.shared_prefix(prompt_len=300, suffix_max=60, prompts=4, samples=8, device="cuda", partition_size=128,
+                           num_heads=32, num_kv_heads=8, head_dim=128, block_size=16)
+    ref, kc, vc, err, _ = run_gpu(pa, step)
+    assert err == 0
+    tables = torch.from_numpy(step.block_tables.astype(np.int32)).cuda()
+    ctx = torch.from_numpy(step.context_lens.astype(np.int32)).cuda()
+    ws = pa.alloc_workspace(step.num_seqs, step.num_heads, step.head_dim,
+                            pa.decode_capacity(tables, step.block_size, 0), step.partition_size, "cuda")
+    kw = dict(partition_size=step.partition_size, workspace=ws)
+    pa.decode(torch.empty_like(ref), step.q, kc, vc, tables, ctx, step.scale, phases=pa.PHASE_PLAN, **kw)
+    for _ in range(2):
+        out = torch.full_like(ref, float("nan"))
+        pa.decode(out, step.q, kc, vc, tables, ctx, step.scale, phases=pa.PHASE_ATTEND, **kw)
+        pa.decode(out, step.q, kc, vc, tables, ctx, step.scale, phases=pa.PHASE_REDUCE, **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+
+
 def test_bad_block_in_a_shared_partition(pa):
     """A block id outside the pool inside a shared partition: flagged, its tokens
     skipped by every sample (their value rows zeroed by the ring's issuer), and

@@ -108,15 +108,25 @@ def test_selftest_host_validation(pa):
 
 def test_workspace_bytes(pa):
     ws = pa.lib.pa_decode_workspace_bytes
-    # one partition: header + work list only (an item is two int32: code and context)
-    assert ws(64, 32, 128, 512, 512) == 256 + 512
-    # several partitions: + (max, sum) and the fp32 partial outputs
-    S, H, D, cap, P = 8, 64, 128, 131072, 512
-    parts = cap // P
     r = lambda n: (n + 255) // 256 * 256  # noqa: E731
-    # header, work list, (max, sum), partial outputs
-    expect = 256 + r(S * parts * 8) + r(S * H * parts * 8) + r(S * H * parts * D * 4)
-    assert ws(S, H, D, cap, P) == expect
+    W, cap_max = 3, 256                    # warps (streams, column groups) and split units
+
+    def expect(S, H, D, cap, P):
+        parts = max(1, -(-cap // P))
+        split = min(cap_max, (S // 2) * parts * H)
+        state = (4 * (D // 16) + 4) * 32 * 4
+        # header; work list (two int32 pairs per item: code, context, split slot, spare),
+        # room for the extra stream items of split shared items; (max, sum) and fp32 partials
+        # when a context spans partitions; split units' stream states and their counters
+        n = 256 + r((S * parts + (W - 1) * split) * 16)
+        if parts > 1:
+            n += r(S * H * parts * 8) + r(S * H * parts * D * 4)
+        return n + r(split * W * W * state) + r(split * 4)
+
+    assert ws(64, 32, 128, 512, 512) == expect(64, 32, 128, 512, 512)
+    assert ws(8, 64, 128, 131072, 512) == expect(8, 64, 128, 131072, 512)
+    assert ws(1, 8, 64, 100, 32) == expect(1, 8, 64, 100, 32)       # one sequence: nothing to split
+    assert ws(1, 8, 64, 100, 32) == 256 + r(1 * 4 * 16) + r(8 * 4 * 8) + r(8 * 4 * 64 * 4)
     assert ws(-1, 1, 64, 10, 512) == 0
     assert ws(1, 1, 64, 10, 0) == 0
 
