@@ -123,45 +123,52 @@ constexpr int PLAN_THREADS = 1024;
 
 // Number of leading whole partitions that sequence s (context c) shares with
 // s + 1 (context c_next): the partitions whose block-table entries name the
-// same physical blocks.  first / first_next are the two tables' first entries
-// (loaded by the caller together with the context lengths, so a pair that
-// shares nothing costs no extra round trip); each compared partition costs one
-// round trip per 16 entries, all issued together.
-__device__ int shared_lead(const DecodeArgs& a, int s, int c, int c_next, int first, int first_next) {
+// same physical blocks.  Called by all lanes of a warp, one sequence each
+// (has_next false past the batch's last pair).  first / first_next are the
+// two tables' first entries, loaded by the caller together with the context
+// lengths, so a pair that shares nothing costs no further load.  The other
+// pairs are compared by the warp together, 32 entries of a partition per
+// round trip: lane j loads entry j of each of the warp's 33 rows (coalesced
+// along the table row) and a pair shares the partition when no lane sees its
+// two rows differ.
+__device__ __forceinline__ int shared_lead(const DecodeArgs& a, int s, bool has_next, int c, int c_next, int first,
+                                           int first_next) {
+    const int lane = threadIdx.x & 31;
     const int P = a.partition_size, bpp = P / a.block_size;
-    const int kmax = min(c, c_next) / P;
-    if (a.pack <= 1 || kmax == 0 || first != first_next) return 0;
-    const int32_t* t0 = table_row(a, s);
-    const int32_t* t1 = table_row(a, s + 1);
-    if (t0 == t1) return kmax;   // two new tokens of one sequence (prefill)
-    int k = 0;
-    for (; k < kmax; ++k) {
-        bool same = true;
-        for (int i0 = 0; i0 < bpp; i0 += 16) {
-            int x[16], y[16];
+    const int kmax = has_next ? min(c, c_next) / P : 0;
+    bool cand = a.pack > 1 && kmax > 0 && first == first_next;
+    int lead = 0;
+    if (cand && table_row(a, s) == table_row(a, s + 1)) {   // two new tokens of one sequence (prefill)
+        lead = kmax;
+        cand = false;
+    }
+    unsigned active = __ballot_sync(FULL_MASK, cand);
+    const int s0 = s - lane;   // the warp's first sequence: pair r is (s0 + r, s0 + r + 1)
+    for (int k = 0; active != 0u; ++k) {
+        // the active pairs share partitions 0 .. k-1 and are compared on partition k
+        unsigned still = active;
+        for (int i0 = 0; i0 < bpp && still != 0u; i0 += 32) {
+            const int j = i0 + lane;
+            const unsigned rows = still | (still << 1);   // row r belongs to pair r or r - 1
+            int e[33];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                if (i0 + j < bpp) {
-                    x[j] = t0[k * bpp + i0 + j];
-                    y[j] = t1[k * bpp + i0 + j];
-                }
+            for (int r = 0; r < 33; ++r) {
+                const bool need = r < 32 ? ((rows >> r) & 1u) != 0u : ((still >> 31) & 1u) != 0u;
+                e[r] = (need && j < bpp) ? table_row(a, s0 + r)[k * bpp + j] : 0;
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (i0 + j < bpp) same &= x[j] == y[j];
+            for (int r = 0; r < 32; ++r) {
+                if ((still >> r) & 1u) {
+                    if (__any_sync(FULL_MASK, j < bpp && e[r] != e[r + 1])) still &= ~(1u << r);
+                }
+            }
         }
-        if (!same) break;
+        if ((still >> lane) & 1u) lead = k + 1;
+        active = still & __ballot_sync(FULL_MASK, k + 1 < kmax);
     }
-    return k;
+    return lead;
 }
 
-// Whole-partition items of sequence s (context c), counted or written to out[].
-// Sequences are packed in runs of up to a.pack, aligned at the start of each
-// chain of consecutive sequences that share their first partition (c0 is the
-// start of s's run) and cut at the chunk's end: for each partition, the run's
-// first sequence emits one item for the run-mates linked to it through that
-// partition (consecutive links); a sequence not covered that way emits its
-// own item.  `lead` holds shared_lead of the sequences from lead_base on.
 // Query columns of a packed item of `count` sequences: it takes the CTA-wide
 // shared layout (several column groups) when they exceed one group of 8.
 __device__ __forceinline__ bool shared_layout(const DecodeArgs& a, int count) { return count * a.group > 8; }
@@ -185,30 +192,28 @@ __device__ int split_candidates(const DecodeArgs& a, int s, int c, const int* le
     return n;
 }
 
-// Whole-partition items of sequence s (context c), counted or written to out[].
-// Sequences are packed in runs of up to a.pack, aligned at the start of each
-// chain of consecutive sequences that share their first partition (c0 is the
-// start of s's run) and cut at the chunk's end: for each partition, the run's
-// first sequence emits one item for the run-mates linked to it through that
-// partition (consecutive links); a sequence not covered that way emits its
-// own item.  A shared-layout item whose number (split_id, counted over the
-// batch) is below a.split_items is emitted as W items, one per stream, that
-// run on different CTAs.  `lead` holds shared_lead of the sequences from
-// lead_base on.
+// Whole-partition items of sequence s (context c) that serve several
+// sequences, counted or written to out[]; *own_from receives the first of the
+// partitions s then reads alone (its own items, one per partition up to
+// c / P, which the caller writes after these).  Sequences are packed in runs
+// of up to a.pack, aligned at the start of each chain of consecutive
+// sequences that share their first partition (c0 is the start of s's run)
+// and cut at the chunk's end: for each partition, the run's first sequence
+// emits one item for the run-mates linked to it through that partition
+// (consecutive links); a sequence not covered that way emits its own item.
+// A shared-layout item whose number (split_id, counted over the batch) is
+// below a.split_items is emitted as W items, one per stream, that run on
+// different CTAs.  `lead` holds shared_lead of the sequences from lead_base on.
 template <bool WRITE>
-__device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base, int c0, int split_id,
-                          int4* out) {
+__device__ __forceinline__ int shared_items(const DecodeArgs& a, int s, int c, const int* lead, int lead_base,
+                                            int c0, int split_id, int4* out, int* own_from) {
     const int nfull = c / a.partition_size, m = a.pack;
-    if (m <= 1) {
-        if (WRITE)
-            for (int k = 0; k < nfull; ++k) out[k] = make_int4(make_item(s, k, 1, a.max_parts), c, -1, 0);
-        return nfull;
-    }
+    *own_from = 0;
+    if (m <= 1) return 0;
     const int end = min(c0 + m, min(a.num_seqs, lead_base + static_cast<int>(blockDim.x)));   // the run: [c0, end)
     if (s == c0) {
         // partitions shared with the next sequence of the run get one item (or
-        // one per stream) for the run-mates linked through them; the rest are
-        // the run start's own
+        // one per stream) for the run-mates linked through them
         const int kshared = s + 1 < end ? min(nfull, lead[s - lead_base]) : 0;
         int n = 0;
         for (int k = 0; k < kshared; ++k) {
@@ -225,17 +230,15 @@ __device__ int full_items(const DecodeArgs& a, int s, int c, const int* lead, in
             if (WRITE) out[n] = make_int4(make_item(s, k, cnt, a.max_parts), c, -1, 0);
             ++n;
         }
-        if (WRITE)
-            for (int k = kshared; k < nfull; ++k) out[n + k - kshared] = make_int4(make_item(s, k, 1, a.max_parts), c, -1, 0);
-        return n + nfull - kshared;
+        *own_from = kshared;
+        return n;
     }
     // a later member is served by the run start's items for the partitions that
-    // every link from c0 to it shares; it emits its own items for the rest
+    // every link from c0 to it shares
     int covered = nfull;
     for (int t = c0; t < s && covered > 0; ++t) covered = min(covered, lead[t - lead_base]);
-    if (WRITE)
-        for (int k = covered; k < nfull; ++k) out[k - covered] = make_int4(make_item(s, k, 1, a.max_parts), c, -1, 0);
-    return nfull - covered;
+    *own_from = covered;
+    return 0;
 }
 
 // Start of s's packing run: runs of a.pack sequences counted from the start of
@@ -255,119 +258,179 @@ __device__ __forceinline__ int run_start(const DecodeArgs& a, int start, const i
 // Ragged tails are emitted longest first, in TAIL_BUCKETS classes of length,
 // so that the units handed out last are the short ones.
 constexpr int TAIL_BUCKETS = 4;
+// Own items a thread writes itself; a longer run of them (long contexts) is
+// written by a whole warp.
+constexpr int OWN_SERIAL = 16;
 
 __device__ __forceinline__ int tail_bucket(int c, int P) {
     const int len = c - (c / P) * P;   // 1..P-1 tokens; 0 for an empty context
     return (len * TAIL_BUCKETS) / P;   // TAIL_BUCKETS - 1 = the longest
 }
 
-__device__ __forceinline__ void plan_body(const DecodeArgs& a) {
-    __shared__ int scratch[33];
-    __shared__ int lead[PLAN_THREADS];
-    if (threadIdx.x == 0) *a.ws_ticket = 0;
+// What a thread knows of its sequence after a chunk's analysis.
+struct PlanSeq {
+    int c;          // clamped context
+    int tb;         // tail class, or -1 (no ragged tail)
+    int c0;         // start of its packing run
+    int sid;        // number of its first split candidate over the batch
+    int nsh;        // shared items it emits
+    int own_from;   // first partition of its own items
+    int ef;         // its first item slot within the chunk's whole-partition items
+    int et;         // its slot within its tail class in the chunk
+};
+
+struct PlanShared {
+    int scratch[33 * (1 + TAIL_BUCKETS)];
+    int lead[PLAN_THREADS];
+    int4 q_range[PLAN_THREADS];   // long own-item runs: (first slot, first partition, count, sequence)
+    int q_ctx[PLAN_THREADS];
+    int q_n;
+};
+
+// Loads and compares the lengths and tables of the chunk of sequences from
+// `start`, then finds each sequence's run, split ids and item counts.
+// tot[0] receives the chunk's whole-partition items, tot[1 + b] its tails of
+// class b; split_total counts split candidates over the chunks so far.
+__device__ __forceinline__ PlanSeq plan_analyse(const DecodeArgs& a, int start, int (&tot)[1 + TAIL_BUCKETS],
+                                                int& split_total, PlanShared& sh) {
     const int P = a.partition_size;
-    // Items: whole partitions first, then one per ragged tail (longest class
-    // first), then nothing else: an empty context is a tail of the shortest
-    // class (its unit writes zeros).  One pass when the batch fits one chunk;
-    // otherwise a counting pass, then a writing pass.
+    const int s = start + threadIdx.x;
+    PlanSeq q{0, -1, s, split_total, 0, 0, 0, 0};
+    __syncthreads();   // the previous chunk's lead[] is no longer read
+    const bool has_next = s + 1 < a.num_seqs;
+    int c_next = 0, first = 0, first_next = 1;
+    if (s < a.num_seqs) {
+        const int raw = a.context_lens[s];
+        const int raw_next = has_next ? a.context_lens[s + 1] : 0;
+        if (a.pack > 1) first = table_row(a, s)[0];
+        if (a.pack > 1 && has_next) first_next = table_row(a, s + 1)[0];
+        q.c = clamp_context(raw, a.cap);
+        c_next = clamp_context(raw_next, a.cap);
+        if (q.c != raw) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
+        if ((q.c % P) != 0 || q.c == 0) q.tb = tail_bucket(q.c, P);
+    }
+    const int l = shared_lead(a, s, has_next, q.c, c_next, first, first_next);
+    sh.lead[threadIdx.x] = l;
+    // without any shared partition in the chunk every sequence is its own run
+    // and nothing is split: two scans fewer
+    if (__syncthreads_or(l > 0)) {
+        q.c0 = run_start(a, start, sh.lead, sh.scratch);
+        int nsplit = 0;
+        q.sid = split_total + cta_exclusive_scan(
+                                  s < a.num_seqs ? split_candidates(a, s, q.c, sh.lead, start, q.c0) : 0, &nsplit,
+                                  sh.scratch);
+        split_total += nsplit;
+        if (s < a.num_seqs) q.nsh = shared_items<false>(a, s, q.c, sh.lead, start, q.c0, q.sid, nullptr, &q.own_from);
+    }
+    int v[1 + TAIL_BUCKETS], ex[1 + TAIL_BUCKETS];
+    v[0] = s < a.num_seqs ? q.nsh + q.c / P - q.own_from : 0;
+#pragma unroll
+    for (int b = 0; b < TAIL_BUCKETS; ++b) v[1 + b] = q.tb == b;
+    cta_exclusive_scan_n<1 + TAIL_BUCKETS>(v, ex, tot, sh.scratch);
+    q.ef = ex[0];
+#pragma unroll
+    for (int b = 0; b < TAIL_BUCKETS; ++b)
+        if (q.tb == b) q.et = ex[1 + b];
+    return q;
+}
+
+// Writes the items of the chunk from `start` (right after its analysis):
+// whole partitions from slot base_full, tails of class b from tail_base[b].
+// A thread writes its sequence's shared items and up to OWN_SERIAL own items;
+// longer runs of own items are queued and written by whole warps.
+__device__ __forceinline__ void plan_write(const DecodeArgs& a, int start, const PlanSeq& q, int base_full,
+                                           const int (&tail_base)[TAIL_BUCKETS], PlanShared& sh) {
+    const int P = a.partition_size;
+    const int s = start + threadIdx.x;
+    if (threadIdx.x == 0) sh.q_n = 0;
+    __syncthreads();
+    if (s < a.num_seqs) {
+        int4* out = a.ws_items + base_full + q.ef;
+        if (q.nsh > 0) {
+            int own_from;
+            shared_items<true>(a, s, q.c, sh.lead, start, q.c0, q.sid, out, &own_from);
+        }
+        const int nown = q.c / P - q.own_from;
+        if (nown <= OWN_SERIAL) {
+            for (int k = 0; k < nown; ++k)
+                out[q.nsh + k] = make_int4(make_item(s, q.own_from + k, 1, a.max_parts), q.c, -1, 0);
+        } else {
+            const int qi = atomicAdd(&sh.q_n, 1);
+            sh.q_range[qi] = make_int4(base_full + q.ef + q.nsh, q.own_from, nown, s);
+            sh.q_ctx[qi] = q.c;
+        }
+        if (q.tb >= 0)
+            a.ws_items[tail_base[q.tb] + q.et] = make_int4(make_item(s, q.c / P, 1, a.max_parts), q.c, -1, 0);
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int nq = sh.q_n;
+    for (int qi = warp; qi < nq; qi += nwarps) {
+        const int4 r = sh.q_range[qi];
+        const int cq = sh.q_ctx[qi];
+        for (int k = lane; k < r.z; k += 32)
+            a.ws_items[r.x + k] = make_int4(make_item(r.w, r.y + k, 1, a.max_parts), cq, -1, 0);
+    }
+}
+
+// The plan itself, run by one CTA.  Items: whole partitions first, then one
+// per ragged tail (longest class first), then nothing else: an empty context
+// is a tail of the shortest class (its unit writes zeros).  One pass when the
+// batch fits one chunk; otherwise a counting pass, then a writing pass.
+__device__ __forceinline__ void plan_body(const DecodeArgs& a) {
+    __shared__ PlanShared sh;
+    if (threadIdx.x == 0) *a.ws_ticket = 0;
     const int CH = blockDim.x;
     const bool one_chunk = a.num_seqs <= CH;
-    int full_total = 0, tail_total[TAIL_BUCKETS] = {0, 0, 0, 0};
-    int c = 0, f = 0, tb = -1, ef = 0, et = 0, sid = 0, split_total = 0;
     // split units' counters start at zero (the last stream of a unit also resets its own)
     for (int i = threadIdx.x; i < a.split_cap; i += blockDim.x) a.ws_split_cnt[i] = 0;
+
+    int split_total = 0;
+    int tot[1 + TAIL_BUCKETS];
+    int full_total = 0, tail_total[TAIL_BUCKETS] = {0, 0, 0, 0};
+    PlanSeq q{};
     for (int start = 0; start < a.num_seqs; start += CH) {
-        const int s = start + threadIdx.x;
-        f = 0;
-        tb = -1;
-        __syncthreads();
-        if (s < a.num_seqs) {
-            const bool has_next = s + 1 < a.num_seqs;
-            const int raw = a.context_lens[s];
-            const int raw_next = has_next ? a.context_lens[s + 1] : 0;
-            const int first = a.pack > 1 ? table_row(a, s)[0] : 0;
-            const int first_next = (a.pack > 1 && has_next) ? table_row(a, s + 1)[0] : 1;
-            c = clamp_context(raw, a.cap);
-            if (c != raw) flag_error(a.dev_err, PA_DEVERR_CONTEXT);
-            lead[threadIdx.x] = shared_lead(a, s, c, clamp_context(raw_next, a.cap), first, first_next);
-            if ((c % P) != 0 || c == 0) tb = tail_bucket(c, P);
-        }
-        __syncthreads();
-        const int c0 = run_start(a, start, lead, scratch);
-        int nsplit = 0;
-        sid = split_total + cta_exclusive_scan(s < a.num_seqs ? split_candidates(a, s, c, lead, start, c0) : 0,
-                                               &nsplit, scratch);
-        split_total += nsplit;
-        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, sid, nullptr);
-        int cf = 0;
-        ef = cta_exclusive_scan(f, &cf, scratch);
-        full_total += cf;
+        q = plan_analyse(a, start, tot, split_total, sh);
+        full_total += tot[0];
 #pragma unroll
-        for (int b = 0; b < TAIL_BUCKETS; ++b) {
-            int cb = 0;
-            const int eb = cta_exclusive_scan(tb == b, &cb, scratch);
-            if (tb == b) et = eb;
-            tail_total[b] += cb;
-        }
+        for (int b = 0; b < TAIL_BUCKETS; ++b) tail_total[b] += tot[1 + b];
     }
     // first slot of each tail class, longest class first
     int tail_base[TAIL_BUCKETS];
-    {
-        int acc = full_total;
+    int acc = full_total;
 #pragma unroll
-        for (int b = TAIL_BUCKETS - 1; b >= 0; --b) {
-            tail_base[b] = acc;
-            acc += tail_total[b];
-        }
-        if (threadIdx.x == 0) *a.ws_count = acc;
+    for (int b = TAIL_BUCKETS - 1; b >= 0; --b) {
+        tail_base[b] = acc;
+        acc += tail_total[b];
     }
+    if (threadIdx.x == 0) *a.ws_count = acc;
     if (one_chunk) {
-        const int s = threadIdx.x;
-        const int c0 = run_start(a, 0, lead, scratch);
-        if (s < a.num_seqs) {
-            full_items<true>(a, s, c, lead, 0, c0, sid, a.ws_items + ef);
-            if (tb >= 0) a.ws_items[tail_base[tb] + et] = make_int4(make_item(s, c / P, 1, a.max_parts), c, -1, 0);
-        }
+        plan_write(a, 0, q, 0, tail_base, sh);
         return;
     }
     int base_full = 0;
     split_total = 0;
     for (int start = 0; start < a.num_seqs; start += CH) {
-        const int s = start + threadIdx.x;
-        f = 0;
-        tb = -1;
-        __syncthreads();
-        if (s < a.num_seqs) {
-            const bool has_next = s + 1 < a.num_seqs;
-            c = clamp_context(a.context_lens[s], a.cap);
-            const int c_next = has_next ? clamp_context(a.context_lens[s + 1], a.cap) : 0;
-            const int first = a.pack > 1 ? table_row(a, s)[0] : 0;
-            const int first_next = (a.pack > 1 && has_next) ? table_row(a, s + 1)[0] : 1;
-            lead[threadIdx.x] = shared_lead(a, s, c, c_next, first, first_next);
-            if ((c % P) != 0 || c == 0) tb = tail_bucket(c, P);
-        }
-        __syncthreads();
-        const int c0 = run_start(a, start, lead, scratch);
-        int nsplit = 0;
-        sid = split_total + cta_exclusive_scan(s < a.num_seqs ? split_candidates(a, s, c, lead, start, c0) : 0,
-                                               &nsplit, scratch);
-        split_total += nsplit;
-        if (s < a.num_seqs) f = full_items<false>(a, s, c, lead, start, c0, sid, nullptr);
-        int chunk_f = 0;
-        ef = cta_exclusive_scan(f, &chunk_f, scratch);
-        if (s < a.num_seqs) full_items<true>(a, s, c, lead, start, c0, sid, a.ws_items + base_full + ef);
+        q = plan_analyse(a, start, tot, split_total, sh);
+        plan_write(a, start, q, base_full, tail_base, sh);
+        base_full += tot[0];
 #pragma unroll
-        for (int b = 0; b < TAIL_BUCKETS; ++b) {
-            int cb = 0;
-            const int eb = cta_exclusive_scan(tb == b, &cb, scratch);
-            if (tb == b) a.ws_items[tail_base[b] + eb] = make_int4(make_item(s, c / P, 1, a.max_parts), c, -1, 0);
-            tail_base[b] += cb;
-        }
-        base_full += chunk_f;
+        for (int b = 0; b < TAIL_BUCKETS; ++b) tail_base[b] += tot[1 + b];
+    }
+}
+
+// Before the wait: the lengths and the first table entries the plan reads
+// (decode rows only; prefill rows find their table through row_seq, which
+// the kernel before this one writes).
+__device__ __forceinline__ void plan_prefetch(const DecodeArgs& a) {
+    for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+        prefetch_l2(a.context_lens + s);
+        if (a.row_seq == nullptr && a.pack > 1) prefetch_l2(a.block_tables + static_cast<size_t>(s) * a.max_blocks);
     }
 }
 
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
+    plan_prefetch(a);
     pdl_wait();
     pdl_launch_dependents();
     plan_body(a);
@@ -378,6 +441,10 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
 // tables, the scatter only the pool, so they need no order between them; the
 // attend kernel that follows waits for both.
 __global__ void __launch_bounds__(PLAN_THREADS) step_prologue_kernel(const DecodeArgs a, const ScatterArgs sa) {
+    if (blockIdx.x == 0)
+        plan_prefetch(a);
+    else
+        scatter_prefetch(sa, static_cast<int>(blockIdx.x) - 1);
     pdl_wait();
     pdl_launch_dependents();
     if (blockIdx.x == 0)
@@ -525,6 +592,10 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         for (int i = 0; i < NS; ++i) mbar_init(smem_u32(&wbars[warp * NS + i]), 1);
     }
     fence_barrier_init();
+    if (tid == 0) {   // lines the plan is writing: warm in L2 when the wait returns
+        prefetch_l2(a.ws_count);
+        prefetch_l2(a.ws_items + blockIdx.x / (a.num_kv_heads * a.head_groups));
+    }
     __syncthreads();
     pdl_wait();               // the work list is written by the plan kernel
     pdl_launch_dependents();
@@ -1048,11 +1119,19 @@ constexpr int REDUCE_HEADS_MAX_PARTS = 32;
 template <int D>
 __global__ void __launch_bounds__(128) reduce_heads_kernel(const DecodeArgs a) {
     constexpr int C4 = D / 4, SUB = 32 / C4, U = 8;   // SUB lanes groups split the partitions
-    pdl_wait();
-    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quads = (a.num_heads + 3) / 4;
     const int s = blockIdx.x / quads, head = (blockIdx.x - (blockIdx.x / quads) * quads) * 4 + warp;
+    if (head < a.num_heads) {   // the lines this warp reads first, while attend finishes
+        const size_t r = static_cast<size_t>(s) * a.num_heads + head;
+        if (lane == 0) prefetch_l2(a.context_lens + s);
+        if (lane == 1) prefetch_l2(a.ws_ml + r * a.max_parts);
+        constexpr int LINES = D / 32;   // 128-byte lines of one partial
+        const int pp = lane / LINES;
+        if (pp < a.max_parts && pp < U) prefetch_l2(a.ws_acc + (r * a.max_parts + pp) * D + (lane % LINES) * 32);
+    }
+    pdl_wait();
+    pdl_launch_dependents();
     const int ctx = clamp_context(a.context_lens[s], a.cap);
     const int nparts = (ctx + a.partition_size - 1) / a.partition_size;
     if (nparts <= 1 || head >= a.num_heads) return;   // single partitions are written by attend
@@ -1115,32 +1194,43 @@ __global__ void __launch_bounds__(128) reduce_heads_kernel(const DecodeArgs a) {
     }
 }
 
-// Longer contexts: one CTA per (seq, head).  The 128 threads are D/4 float4
-// columns x G partition groups (group g takes partitions g, g+G, ...); the
-// groups are combined in a fixed order.
+// Longer contexts: one CTA of REDUCE_PARTS_THREADS per (seq, head).  The
+// threads are D/4 float4 columns x G partition groups (group g takes
+// partitions g, g+G, ...); the groups are combined in a fixed order.  The
+// context length and the first REDUCE_PARTS_THREADS (max, sum) pairs are
+// loaded in one round trip.
+constexpr int REDUCE_PARTS_THREADS = 256;
+
 template <int D>
-__global__ void __launch_bounds__(128) reduce_parts_kernel(const DecodeArgs a) {
-    constexpr int C4 = D / 4, G = 128 / C4, U = 8;
-    __shared__ float red[4];
+__global__ void __launch_bounds__(REDUCE_PARTS_THREADS, 4) reduce_parts_kernel(const DecodeArgs a) {
+    constexpr int T = REDUCE_PARTS_THREADS, C4 = D / 4, G = T / C4, U = 8;
+    __shared__ float red[T / 32];
     __shared__ float4 so[G][C4];
     __shared__ float sl[G];
-    pdl_wait();
-    pdl_launch_dependents();
     const int tid = threadIdx.x;
     const int s = blockIdx.x / a.num_heads, head = blockIdx.x - (blockIdx.x / a.num_heads) * a.num_heads;
-    const int ctx = clamp_context(a.context_lens[s], a.cap);
-    const int nparts = (ctx + a.partition_size - 1) / a.partition_size;
-    if (nparts <= 1) return;   // written by the attend kernel
     const size_t row = static_cast<size_t>(s) * a.num_heads + head;
+    // the lines this CTA reads first, while attend finishes
+    if (tid == 0) prefetch_l2(a.context_lens + s);
+    if (tid < a.max_parts && (tid & 15) == 0) prefetch_l2(a.ws_ml + row * a.max_parts + tid);
+    pdl_wait();
+    pdl_launch_dependents();
     const float2* mlp = a.ws_ml + row * a.max_parts;
     const float4* accp = reinterpret_cast<const float4*>(a.ws_acc + row * a.max_parts * D);
-    float M = NEG_INF;
-    for (int p = tid; p < nparts; p += 128) M = fmaxf(M, mlp[p].x);
+    const int raw = a.context_lens[s];
+    const float m_any = tid < a.max_parts ? mlp[tid].x : NEG_INF;
+    const int ctx = clamp_context(raw, a.cap);
+    const int nparts = (ctx + a.partition_size - 1) / a.partition_size;
+    if (nparts <= 1) return;   // written by the attend kernel
+    float M = tid < nparts ? m_any : NEG_INF;
+    for (int p = tid + T; p < nparts; p += T) M = fmaxf(M, mlp[p].x);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
     if ((tid & 31) == 0) red[tid >> 5] = M;
     __syncthreads();
-    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    M = red[0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) M = fmaxf(M, red[w]);
     const int c4 = tid % C4, g = tid / C4;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     float L = 0.f;
@@ -1172,7 +1262,7 @@ __global__ void __launch_bounds__(128) reduce_parts_kernel(const DecodeArgs a) {
     so[g][c4] = o;
     if (c4 == 0) sl[g] = L;
     __syncthreads();
-    for (int d = tid; d < D; d += 128) {
+    for (int d = tid; d < D; d += T) {
         float O = 0.f, Lt = 0.f;
 #pragma unroll
         for (int k = 0; k < G; ++k) {
@@ -1462,8 +1552,9 @@ static int decode_impl(void* out, pa_dtype out_dtype, const void* q, const void*
         } else {
             const long long rows = static_cast<long long>(num_seqs) * num_heads;
             if (rows > INT_MAX) return PA_ERR_UNSUPPORTED;
-            e = head_dim == 128 ? launch_pdl(reduce_parts_kernel<128>, dim3(rows), dim3(128), 0, st, a)
-                                : launch_pdl(reduce_parts_kernel<64>, dim3(rows), dim3(128), 0, st, a);
+            e = head_dim == 128
+                    ? launch_pdl(reduce_parts_kernel<128>, dim3(rows), dim3(REDUCE_PARTS_THREADS), 0, st, a)
+                    : launch_pdl(reduce_parts_kernel<64>, dim3(rows), dim3(REDUCE_PARTS_THREADS), 0, st, a);
         }
         if (launch_status(e) != PA_OK) return PA_ERR_CUDA;
     }

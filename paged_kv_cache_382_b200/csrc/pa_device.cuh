@@ -37,8 +37,17 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 // Waits until the kernel this one depends on (the previous one in the stream)
 // has completed and its memory is visible; a no-op when launched normally.
-// Every CTA calls it before its first access to global memory.
+// Every CTA calls it before its first load or store of global memory.  Before
+// it a CTA may only issue L2 prefetches (prefetch_l2) of addresses it computes
+// without loading anything: a prefetch returns no data and L2 is coherent, so
+// a line the previous kernel still writes is simply updated in L2, while the
+// address translation and the line are warm when the wait returns.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Brings the line holding p into L2 (and its translation into the TLBs).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
 
 // Lets the next kernel in the stream begin launching (its CTAs then wait in
 // pdl_wait until this grid completes).
@@ -180,6 +189,56 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* total, int* scratc
     __syncthreads();
     *total = scratch[32];
     return scratch[warp] + inc - v;
+}
+
+// N exclusive prefix sums over the CTA in one pass (one set of barriers for all
+// N values): ex[i] receives the sum of v[i] over the lower threads, total[i]
+// the sum over the CTA.  `scratch` holds 33 * N ints.
+template <int N>
+__device__ __forceinline__ void cta_exclusive_scan_n(const int (&v)[N], int (&ex)[N], int (&total)[N],
+                                                     int* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int inc[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) inc[i] = v[i];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const int n = __shfl_up_sync(FULL_MASK, inc[i], o);
+            if (lane >= o) inc[i] += n;
+        }
+    }
+    __syncthreads();
+    if (lane == 31) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) scratch[i * 33 + warp] = inc[i];
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int x[N], xi[N];
+#pragma unroll
+        for (int i = 0; i < N; ++i) xi[i] = x[i] = lane < nw ? scratch[i * 33 + lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int n = __shfl_up_sync(FULL_MASK, xi[i], o);
+                if (lane >= o) xi[i] += n;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            if (lane < nw) scratch[i * 33 + lane] = xi[i] - x[i];
+            if (lane == 31) scratch[i * 33 + 32] = xi[i];
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        total[i] = scratch[i * 33 + 32];
+        ex[i] = scratch[i * 33 + warp] + inc[i] - v[i];
+    }
 }
 
 __device__ __forceinline__ int warp_inclusive_max_scan(int v) {

@@ -21,25 +21,55 @@ struct ScatterArgs {
 
 // Token t goes to block slot / B at offset slot % B, for every kv head; a
 // negative slot writes nothing, a slot past the pool is flagged and skipped.
-// The CTA's threads stride over the token's Hkv x row_vecs vectors.
-__device__ __forceinline__ void scatter_token(const ScatterArgs& s, int t) {
-    const int64_t slot = s.slot_mapping[t];
-    if (slot < 0) return;
-    if (slot >= s.num_slots) {
-        if (threadIdx.x == 0) flag_error(s.dev_err, PA_DEVERR_SLOT);
-        return;
+// The CTA's threads stride over the token's Hkv x row_vecs vectors.  Each
+// thread loads up to SCATTER_BATCH vectors of K and of V before it stores
+// any, and the first batch is loaded together with the slot (the source rows
+// exist whatever the slot says), so a token costs one round trip per batch.
+constexpr int SCATTER_BATCH = 4;
+
+// Before the wait of the launch: token t's slot and source rows into L2.
+__device__ __forceinline__ void scatter_prefetch(const ScatterArgs& s, int t) {
+    const int per_token = s.num_kv_heads * s.row_vecs;
+    if (threadIdx.x == 0) prefetch_l2(s.slot_mapping + t);
+    for (int i = threadIdx.x * 8; i < per_token; i += blockDim.x * 8) {   // one 128-byte line per 8 vectors
+        prefetch_l2(s.key + static_cast<int64_t>(t) * per_token + i);
+        prefetch_l2(s.value + static_cast<int64_t>(t) * per_token + i);
     }
-    const int64_t block = slot / s.block_size;
-    const int offset = static_cast<int>(slot - block * s.block_size);
+}
+
+__device__ __forceinline__ void scatter_token(const ScatterArgs& s, int t) {
     const int per_token = s.num_kv_heads * s.row_vecs;
     const uint4* ksrc = s.key + static_cast<int64_t>(t) * per_token;
     const uint4* vsrc = s.value + static_cast<int64_t>(t) * per_token;
-    for (int i = threadIdx.x; i < per_token; i += blockDim.x) {
-        const int h = i / s.row_vecs;
-        const int v = i - h * s.row_vecs;
-        const int64_t dst = ((block * s.num_kv_heads + h) * s.block_size + offset) * s.row_vecs + v;
-        s.k_cache[dst] = ksrc[i];
-        s.v_cache[dst] = vsrc[i];
+    const int64_t slot = s.slot_mapping[t];
+    for (int i0 = threadIdx.x; i0 < per_token; i0 += SCATTER_BATCH * blockDim.x) {
+        uint4 kv[SCATTER_BATCH], vv[SCATTER_BATCH];
+#pragma unroll
+        for (int u = 0; u < SCATTER_BATCH; ++u) {
+            const int i = i0 + u * blockDim.x;
+            if (i < per_token) {
+                kv[u] = ksrc[i];
+                vv[u] = vsrc[i];
+            }
+        }
+        if (slot < 0) return;
+        if (slot >= s.num_slots) {
+            if (threadIdx.x == 0) flag_error(s.dev_err, PA_DEVERR_SLOT);
+            return;
+        }
+        const int64_t block = slot / s.block_size;
+        const int offset = static_cast<int>(slot - block * s.block_size);
+#pragma unroll
+        for (int u = 0; u < SCATTER_BATCH; ++u) {
+            const int i = i0 + u * blockDim.x;
+            if (i < per_token) {
+                const int h = i / s.row_vecs;
+                const int v = i - h * s.row_vecs;
+                const int64_t dst = ((block * s.num_kv_heads + h) * s.block_size + offset) * s.row_vecs + v;
+                s.k_cache[dst] = kv[u];
+                s.v_cache[dst] = vv[u];
+            }
+        }
     }
 }
 
