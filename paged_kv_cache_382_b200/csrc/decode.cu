@@ -1122,13 +1122,15 @@ __global__ void __launch_bounds__(128) reduce_heads_kernel(const DecodeArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quads = (a.num_heads + 3) / 4;
     const int s = blockIdx.x / quads, head = (blockIdx.x - (blockIdx.x / quads) * quads) * 4 + warp;
-    if (head < a.num_heads) {   // the lines this warp reads first, while attend finishes
+    if (head < a.num_heads) {   // the lines this warp reads first, while attend finishes: the length,
+        // the (max, sum) pairs and the first two partials (every row the kernel merges has at least two;
+        // how many more is known only from the length)
         const size_t r = static_cast<size_t>(s) * a.num_heads + head;
         if (lane == 0) prefetch_l2(a.context_lens + s);
         if (lane == 1) prefetch_l2(a.ws_ml + r * a.max_parts);
         constexpr int LINES = D / 32;   // 128-byte lines of one partial
         const int pp = lane / LINES;
-        if (pp < a.max_parts && pp < U) prefetch_l2(a.ws_acc + (r * a.max_parts + pp) * D + (lane % LINES) * 32);
+        if (pp < 2 && pp < a.max_parts) prefetch_l2(a.ws_acc + (r * a.max_parts + pp) * D + (lane % LINES) * 32);
     }
     pdl_wait();
     pdl_launch_dependents();
