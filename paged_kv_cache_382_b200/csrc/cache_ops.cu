@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const ScatterArg
 }
 
 // grid.y = pair index; grid.x CTAs stride over the block's 16-byte vectors.
+constexpr int COPY_BATCH = 4;
 __global__ void __launch_bounds__(256)
 copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                    const int64_t* __restrict__ pairs, int64_t block_vecs, int num_blocks,
@@ -38,12 +39,28 @@ copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
     const uint4* vs = v_cache + src * block_vecs;
     uint4* kd = k_cache + dst * block_vecs;
     uint4* vd = v_cache + dst * block_vecs;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < block_vecs;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const uint4 a = ks[i];
-        const uint4 b = vs[i];
-        kd[i] = a;
-        vd[i] = b;
+    // each thread loads COPY_BATCH vectors of K and of V before it stores any
+    // (one round trip per batch; the launch sizes the grid for one batch)
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < block_vecs;
+         i0 += COPY_BATCH * stride) {
+        uint4 a[COPY_BATCH], b[COPY_BATCH];
+#pragma unroll
+        for (int u = 0; u < COPY_BATCH; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < block_vecs) {
+                a[u] = ks[i];
+                b[u] = vs[i];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < COPY_BATCH; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < block_vecs) {
+                kd[i] = a[u];
+                vd[i] = b[u];
+            }
+        }
     }
 }
 
@@ -121,7 +138,7 @@ extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_d
     if (num_pairs > 65535) return PA_ERR_UNSUPPORTED;   // grid.y limit
     const int64_t block_vecs = static_cast<int64_t>(block_bytes / 16);
     const int threads = 256;
-    int64_t ctas = (block_vecs + threads * 4 - 1) / (threads * 4);
+    int64_t ctas = (block_vecs + threads * COPY_BATCH - 1) / (threads * COPY_BATCH);
     if (ctas < 1) ctas = 1;
     if (ctas > 1024) ctas = 1024;
     dim3 grid(static_cast<unsigned>(ctas), static_cast<unsigned>(num_pairs));

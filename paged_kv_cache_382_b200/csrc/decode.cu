@@ -86,7 +86,7 @@ struct DecodeArgs {
     int head_groups;     // ceil(group / 8): units per kv head
     float scale_log2;    // scale * log2(e)
     int out_f32;         // 1: out is fp32, 0: out is bf16
-    int pack;            // sequences a packed item may serve (32 / group; 1 = no packing)
+    int pack;            // sequences a packed item may serve (8 * ATTEND_WARPS / group; 1 = no packing)
     const int32_t* row_seq;   // prefill: the sequence (block-table row) of each query row; null = identity
 };
 
