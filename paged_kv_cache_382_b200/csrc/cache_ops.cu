@@ -120,6 +120,7 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
     sa.block_size = block_size;
     sa.num_slots = num_slots;
     sa.dev_err = dev_err;
+    sa.after_copies = 0;
     if (const int rc = device_check(k_cache)) return rc;
     return launch_status(launch_pdl(reshape_and_cache_kernel, dim3(num_tokens), dim3(threads), 0,
                                     as_stream(stream), sa));

@@ -445,7 +445,11 @@ __global__ void __launch_bounds__(PLAN_THREADS) step_prologue_kernel(const Decod
         plan_prefetch(a);
     else
         scatter_prefetch(sa, static_cast<int>(blockIdx.x) - 1);
-    pdl_wait();
+    // Right after this call's own block-copy kernel the plan need not wait: this
+    // launch begins only once every copy CTA has passed its own wait (all work
+    // before the call complete and visible), and the copies touch only the pool,
+    // which the plan does not read.  The scatter writes into copied blocks: it waits.
+    if (blockIdx.x != 0 || !sa.after_copies) pdl_wait();
     pdl_launch_dependents();
     if (blockIdx.x == 0)
         plan_body(a);
@@ -1673,6 +1677,7 @@ extern "C" int pa_decode_step(void* out, pa_dtype out_dtype, const void* q, cons
     sa.block_size = block_size;
     sa.num_slots = static_cast<int64_t>(num_blocks) * block_size;
     sa.dev_err = dev_err;
+    sa.after_copies = num_pairs > 0 ? 1 : 0;   // the copy kernel is launched right before the prologue
     const size_t block_bytes = static_cast<size_t>(num_kv_heads) * block_size * head_dim * element_bytes(dtype);
     // copy-on-write copies first (the writes may land in the copied blocks)
     auto copies = [=](cudaStream_t, int) {

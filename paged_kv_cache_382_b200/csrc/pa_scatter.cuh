@@ -17,6 +17,7 @@ struct ScatterArgs {
     int num_kv_heads, row_vecs, block_size;
     int64_t num_slots;         // NB * B
     int32_t* dev_err;
+    int after_copies;          // 1: the launch follows this call's own block-copy kernel
 };
 
 // Token t goes to block slot / B at offset slot % B, for every kv head; a
