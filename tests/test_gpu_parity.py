@@ -560,6 +560,38 @@ def random_fork_step(seed, Hq, Hkv, d, B, P, adjacent=True):
         slot_mapping=np.full(S, -1, dtype=np.int64), copy_pairs=np.zeros((0, 2), dtype=np.int64))
 
 
+@pytest.mark.parametrize("heads,B", [((32, 8), 16), ((8, 8), 4), ((64, 8), 8)], ids=["g4_b16", "g1_b4", "g8_b8"])
+def test_short_tails_and_batch_order(pa, heads, B):
+    """Ragged tails of every length class, single-tile ones and empty contexts
+    included, at block sizes 16, 4 and 8: against the oracle, and independent
+    of the batch around them: the batch reversed, and with one sequence dropped
+    (other units around each tail, other unit counts per class), gives every
+    remaining row bit for bit."""
+    Hq, Hkv = heads
+    P = 64
+    rng = np.random.default_rng(11)
+    rests = [0, 1, 5, 9, 16, 17, 30, 63]
+    ctx = [int(P * rng.integers(0, 4) + rests[i % len(rests)]) for i in range(26)]
+    ctx[3] = 0
+    step = W.independent("single_tile_tails", ctx, num_heads=Hq, num_kv_heads=Hkv, block_size=B, seed=5,
+                         device="cuda", partition_size=P)
+    out, *_, err, _ = run_gpu(pa, step, out_dtype=torch.bfloat16)
+    assert err == 0
+    assert_close(f64(out), full_oracle(step), torch.bfloat16, torch.bfloat16, "single-tile tails")
+    S = step.num_seqs
+    for order in (list(range(S - 1, -1, -1)), [i for i in range(S) if i != 7]):
+        other = W.DecodeStep(**{**step.__dict__})
+        other.q = step.q[order].contiguous()
+        other.block_tables = step.block_tables[order]
+        other.context_lens = step.context_lens[order]
+        other.slot_mapping = step.slot_mapping[order]
+        other.new_key = step.new_key[order].contiguous()
+        other.new_value = step.new_value[order].contiguous()
+        out2, *_, err2, _ = run_gpu(pa, other, out_dtype=torch.bfloat16)
+        assert err2 == 0
+        assert torch.equal(out2, out[order])
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2, 3])
 @pytest.mark.parametrize("heads", [(16, 4), (8, 4), (8, 8)], ids=["g4", "g2", "g1"])
 def test_random_fork_histories(pa, seed, heads):
