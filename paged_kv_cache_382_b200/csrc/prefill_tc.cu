@@ -333,8 +333,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             }
         } else if (compute_warp) {
             // Q tile: row r = new token tok0 + r / G, head kvh * G + r % G; rows past
-            // the unit's tokens are zero.  All loads are issued before the first
-            // store (one round trip), in two batches to bound the registers.
+            // the unit's tokens are zero.  A thread's loads go out in batches of
+            // up to eight, each batch issued together before its stores (the
+            // batch size bounds the registers the loads hold).
             constexpr int QLOADS = TC_ROWS * (D / 8) / (TC_COMPUTE_WARPS * 32);
             constexpr int QBATCH = QLOADS < 8 ? QLOADS : 8;
 #pragma unroll
